@@ -1,0 +1,224 @@
+"""ctypes binding of libdynrad.so (declared in include/dynrad.h).
+
+Argument marshalling only: tensors become device pointers, the stream is
+torch's current stream, every step of the path runs in the library's kernels.
+There is no fallback: if the library is missing or fails to load, every call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdynrad.so")
+
+DYNRAD_OK = 0
+DYNRAD_ERR_INVALID_ARG = 1
+DYNRAD_ERR_UNSUPPORTED = 2
+DYNRAD_ERR_CAPACITY = 3
+DYNRAD_ERR_CUDA = 4
+DYNRAD_ERR_DEVICE = 5
+
+DYNRAD_STATIC_RATIO = 0
+DYNRAD_DYNAMIC_THRESHOLD = 1
+MODES = {"static": DYNRAD_STATIC_RATIO, "dynamic": DYNRAD_DYNAMIC_THRESHOLD}
+
+# every extern "C" symbol include/dynrad.h declares
+EXPORTED = (
+    "dynrad_num_blocks",
+    "dynrad_build_candidates",
+    "dynrad_select_workspace_bytes",
+    "dynrad_select_blocks",
+    "dynrad_sparse_attn",
+    "dynrad_device_status",
+    "dynrad_status_string",
+)
+
+
+class DynradGeom(ctypes.Structure):
+    _fields_ = [
+        ("frames", ctypes.c_int32),
+        ("height", ctypes.c_int32),
+        ("width", ctypes.c_int32),
+        ("block", ctypes.c_int32),
+        ("gamma", ctypes.c_double),
+        ("lambda_", ctypes.c_double),
+        ("theta_c", ctypes.c_double),
+        ("theta_m", ctypes.c_double),
+        ("eps", ctypes.c_double),
+        ("force_t", ctypes.c_int32),
+    ]
+
+
+class DynradError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+_VP = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+_I64P = ctypes.POINTER(ctypes.c_int64)
+_I32P = ctypes.POINTER(ctypes.c_int32)
+_GP = ctypes.POINTER(DynradGeom)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library.  Raises if libdynrad.so is absent (no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m block_sparse_attention_candidate_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        L.dynrad_num_blocks.restype = _I64
+        L.dynrad_num_blocks.argtypes = [_GP]
+        L.dynrad_build_candidates.restype = ctypes.c_int
+        L.dynrad_build_candidates.argtypes = [_GP, _VP, _VP, _I64, _VP, _VP, _I64P, _I64P, _VP]
+        L.dynrad_select_workspace_bytes.restype = _SZ
+        L.dynrad_select_workspace_bytes.argtypes = [_I32, _I32, _I32, _I32, _GP, _I64]
+        L.dynrad_select_blocks.restype = ctypes.c_int
+        L.dynrad_select_blocks.argtypes = [_VP, _VP, _I32, _I32, _I32, _I32, _GP, _VP, _VP, _I64, _I64,
+                                           _VP, _VP, _I32, ctypes.c_double, _VP, _VP, _I64, _VP, _VP, _SZ,
+                                           _VP]
+        L.dynrad_sparse_attn.restype = ctypes.c_int
+        L.dynrad_sparse_attn.argtypes = [_VP, _VP, _VP, _I32, _I32, _I32, _I32, _I32, _VP, _VP,
+                                         ctypes.c_float, _VP, _VP, _VP]
+        L.dynrad_device_status.restype = ctypes.c_int
+        L.dynrad_device_status.argtypes = [_I32P, _I32, _VP]
+        L.dynrad_status_string.restype = ctypes.c_char_p
+        L.dynrad_status_string.argtypes = [_I32]
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().dynrad_status_string(int(status)).decode()
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != DYNRAD_OK:
+        raise DynradError(rc, where)
+
+
+def make_geom(g) -> DynradGeom:
+    """C geometry struct from an object with frames, height, width, block,
+    gamma, lam, theta_c, theta_m, eps, force_t (workloads.Geometry)."""
+    return DynradGeom(int(g.frames), int(g.height), int(g.width), int(g.block), float(g.gamma),
+                      float(g.lam), float(g.theta_c), float(g.theta_m), float(g.eps), int(g.force_t))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def dynrad_num_blocks(geom) -> int:
+    return int(lib().dynrad_num_blocks(ctypes.byref(make_geom(geom))))
+
+
+def dynrad_build_candidates(geom, device=None, stream=None) -> dict:
+    """Stage 1.  Returns dict(row_ptr, col, forced_lo, forced_hi: int32 CUDA
+    tensors; nnz, max_row: ints).  Synchronizes once (size query)."""
+    L = lib()
+    cg = make_geom(geom)
+    nb = int(L.dynrad_num_blocks(ctypes.byref(cg)))
+    if nb <= 0:
+        raise DynradError(DYNRAD_ERR_INVALID_ARG, "dynrad_build_candidates")
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    row_ptr = torch.empty(nb + 1, dtype=torch.int32, device=device)
+    flo = torch.empty(nb, dtype=torch.int32, device=device)
+    fhi = torch.empty(nb, dtype=torch.int32, device=device)
+    nnz = ctypes.c_int64(0)
+    mx = ctypes.c_int64(0)
+    st = _stream(stream)
+    _check(L.dynrad_build_candidates(ctypes.byref(cg), _ptr(row_ptr), None, 0, _ptr(flo), _ptr(fhi),
+                                     ctypes.byref(nnz), ctypes.byref(mx), st), "dynrad_build_candidates")
+    col = torch.empty(max(1, nnz.value), dtype=torch.int32, device=device)
+    _check(L.dynrad_build_candidates(ctypes.byref(cg), _ptr(row_ptr), _ptr(col), col.numel(), _ptr(flo),
+                                     _ptr(fhi), ctypes.byref(nnz), ctypes.byref(mx), st),
+           "dynrad_build_candidates")
+    return {"row_ptr": row_ptr, "col": col[: nnz.value], "forced_lo": flo, "forced_hi": fhi,
+            "nnz": nnz.value, "max_row": mx.value, "nb": nb}
+
+
+def dynrad_select_workspace_bytes(B, H, N, D, geom, cand_nnz) -> int:
+    return int(lib().dynrad_select_workspace_bytes(B, H, N, D, ctypes.byref(make_geom(geom)), cand_nnz))
+
+
+class SelectBuffers:
+    """Caller-owned outputs and workspace of dynrad_select_blocks (reusable)."""
+
+    def __init__(self, B, H, N, D, geom, cand, device=None, scores=False):
+        device = device or torch.device("cuda", torch.cuda.current_device())
+        nb = cand["nb"]
+        ws = dynrad_select_workspace_bytes(B, H, N, D, geom, cand["nnz"])
+        if ws == 0:
+            raise DynradError(DYNRAD_ERR_INVALID_ARG, "dynrad_select_workspace_bytes")
+        self.workspace = torch.empty(ws + 256, dtype=torch.uint8, device=device)
+        off = (-self.workspace.data_ptr()) % 256
+        self.ws_view = self.workspace[off:off + ws]
+        self.row_ptr = torch.empty(B * H * nb + 1, dtype=torch.int32, device=device)
+        self.col_idx = torch.empty(B * H * cand["nnz"], dtype=torch.int32, device=device)
+        self.scores = torch.empty(B * H * cand["nnz"], dtype=torch.float32, device=device) if scores else None
+
+
+def dynrad_select_blocks(q, k, geom, cand, mode, value, scores=False, buffers=None, stream=None):
+    """Stage 2.  q, k: bf16 [B, H, N, D] CUDA.  Returns (row_ptr, col_idx,
+    scores or None); col_idx has capacity B*H*cand_nnz (use row_ptr[-1])."""
+    _require_cuda(q, k)
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16:
+        raise ValueError("q, k must be bf16")
+    B, H, N, D = q.shape
+    buf = buffers or SelectBuffers(B, H, N, D, geom, cand, q.device, scores)
+    if scores and buf.scores is None:
+        raise ValueError("buffers were made without a score array")
+    L = lib()
+    cg = make_geom(geom)
+    _check(L.dynrad_select_blocks(_ptr(q), _ptr(k), B, H, N, D, ctypes.byref(cg), _ptr(cand["row_ptr"]),
+                                  _ptr(cand["col"]), cand["nnz"], cand["max_row"], _ptr(cand["forced_lo"]),
+                                  _ptr(cand["forced_hi"]), MODES[mode] if isinstance(mode, str) else mode,
+                                  float(value), _ptr(buf.row_ptr), _ptr(buf.col_idx), buf.col_idx.numel(),
+                                  _ptr(buf.scores) if scores else None, _ptr(buf.ws_view),
+                                  buf.ws_view.numel(), _stream(stream)),
+           "dynrad_select_blocks")
+    return buf.row_ptr, buf.col_idx, (buf.scores if scores else None)
+
+
+def dynrad_sparse_attn(q, k, v, block, row_ptr, col_idx, scale=0.0, out=None, lse=None, stream=None):
+    """Stage 3.  q, k, v: bf16 [B, H, N, D] CUDA; CSR over B*H*Nb rows.
+    Returns (o bf16 [B, H, N, D], lse fp32 [B, H, N])."""
+    _require_cuda(q, k, v, row_ptr, col_idx)
+    B, H, N, D = q.shape
+    o = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(lib().dynrad_sparse_attn(_ptr(q), _ptr(k), _ptr(v), B, H, N, D, int(block), _ptr(row_ptr),
+                                    _ptr(col_idx), float(scale), _ptr(o), _ptr(lse_t), _stream(stream)),
+           "dynrad_sparse_attn")
+    return o, lse_t
+
+
+def dynrad_device_status(clear: bool = True, stream=None) -> int:
+    v = ctypes.c_int32(0)
+    _check(lib().dynrad_device_status(ctypes.byref(v), 1 if clear else 0, _stream(stream)),
+           "dynrad_device_status")
+    return int(v.value)

@@ -1,0 +1,362 @@
+// C ABI of the DynamicRad hot path (declared in include/dynrad.h).
+//
+// Host side only: argument checks, launch configuration, TMA descriptor
+// encoding.  Every arithmetic step of the path runs in the kernels included
+// below.
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "attention.cuh"
+#include "candidates.cuh"
+#include "common.cuh"
+#include "select.cuh"
+
+using namespace dynrad;
+
+namespace {
+
+constexpr int kMaxFrames = 16384;
+constexpr int kMaxBlocks = 16384;    // Nb bound of the selection kernel's shared memory
+
+inline cudaStream_t as_stream(dynrad_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? DYNRAD_OK : DYNRAD_ERR_CUDA;
+}
+
+// Shared geometry validation; fills the device struct.
+int check_geom(const dynrad_geom* g, GeomDev* out) {
+  if (g == nullptr) return DYNRAD_ERR_INVALID_ARG;
+  if (g->frames < 1 || g->height < 1 || g->width < 1 || g->block < 1) return DYNRAD_ERR_INVALID_ARG;
+  if (!(g->gamma > 0.0) || !(g->lambda > 0.0) || !(g->eps >= 0.0)) return DYNRAD_ERR_INVALID_ARG;
+  if (!std::isfinite(g->gamma) || !std::isfinite(g->lambda) || !std::isfinite(g->eps))
+    return DYNRAD_ERR_INVALID_ARG;
+  if (!(g->theta_c >= 0.0 && g->theta_c <= 1.0) || !(g->theta_m >= 0.0 && g->theta_m <= 1.0))
+    return DYNRAD_ERR_INVALID_ARG;
+  if (g->force_t < 0 || g->force_t > 1) return DYNRAD_ERR_INVALID_ARG;
+  const int64_t nt = static_cast<int64_t>(g->height) * g->width;
+  const int64_t n = nt * g->frames;
+  if (nt > INT32_MAX / 4 || n > INT32_MAX / 2) return DYNRAD_ERR_UNSUPPORTED;
+  if (g->frames > kMaxFrames) return DYNRAD_ERR_UNSUPPORTED;
+  const int64_t nb = (n + g->block - 1) / g->block;
+  if (out != nullptr) {
+    out->frames = g->frames;
+    out->nt = static_cast<int32_t>(nt);
+    out->block = g->block;
+    out->nb = static_cast<int32_t>(nb);
+    out->n = static_cast<int32_t>(n);
+    out->force_t = g->force_t;
+    int64_t l0 = 1;
+    while (l0 < nt) l0 <<= 1;  // Eq. 1: smallest power of two >= N_t
+    out->l0 = l0;
+    out->gamma = g->gamma;
+    out->lambda = g->lambda;
+    out->theta_c = g->theta_c;
+    out->theta_m = g->theta_m;
+    out->eps = g->eps;
+  }
+  return DYNRAD_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct SelectWorkspace {
+  size_t qbar, kbar, kept, partial, total;
+};
+
+SelectWorkspace select_layout(int64_t bh, int64_t nb, int64_t d, int64_t cand_nnz) {
+  SelectWorkspace w;
+  const int64_t rows = bh * nb;
+  const int64_t tiles = (rows + 1 + kScanTile - 1) / kScanTile;
+  w.qbar = 0;
+  w.kbar = align256(w.qbar + static_cast<size_t>(rows * d) * 4);
+  w.kept = align256(w.kbar + static_cast<size_t>(rows * d) * 4);
+  w.partial = align256(w.kept + static_cast<size_t>(bh * cand_nnz) * 4);
+  w.total = align256(w.partial + static_cast<size_t>(tiles) * 8);
+  return w;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 3-D map over a [BH, N, D] bf16 tensor: box = 64 columns (128 B) x rows x 1,
+// 128-byte swizzle; rows past N of a head read as zeros.
+bool encode_map(CUtensorMap* map, const void* base, int D, int N, int BH, int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(N) * D * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                         strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, int BS>
+int launch_attn(const void* q, const void* k, const void* v, int BH, int N, const int32_t* row_ptr,
+                const int32_t* col_idx, float scale, void* o, float* lse, cudaStream_t st) {
+  using C = AttnCfg<D, BS>;
+  CUtensorMap mq, mk, mv;
+  if (!encode_map(&mq, q, D, N, BH, 128) || !encode_map(&mk, k, D, N, BH, BS) ||
+      !encode_map(&mv, v, D, N, BH, BS))
+    return DYNRAD_ERR_CUDA;
+  static bool attr_set = false;  // per instantiation
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(sparse_attn_kernel<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemTotal) != cudaSuccess)
+      return DYNRAD_ERR_CUDA;
+    attr_set = true;
+  }
+  AttnParams p;
+  p.row_ptr = row_ptr;
+  p.col_idx = col_idx;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.N = N;
+  p.nb = (N + BS - 1) / BS;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int tiles = (p.nb + C::kR - 1) / C::kR;
+  dim3 grid(tiles, BH);
+  sparse_attn_kernel<D, BS><<<grid, 192, C::kSmemTotal, st>>>(mq, mk, mv, p);
+  return launch_status();
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int64_t dynrad_num_blocks(const dynrad_geom* geom) {
+  GeomDev g;
+  if (check_geom(geom, &g) != DYNRAD_OK) return 0;
+  return g.nb;
+}
+
+const char* dynrad_status_string(int32_t status) {
+  switch (status) {
+    case DYNRAD_OK: return "ok";
+    case DYNRAD_ERR_INVALID_ARG: return "invalid argument";
+    case DYNRAD_ERR_UNSUPPORTED: return "unsupported size or parameter";
+    case DYNRAD_ERR_CAPACITY: return "output or workspace capacity exceeded";
+    case DYNRAD_ERR_CUDA: return "CUDA runtime error";
+    case DYNRAD_ERR_DEVICE: return "device-side check or bounded wait failed";
+    default: return "unknown status";
+  }
+}
+
+int dynrad_device_status(int32_t* status_out, int32_t clear, dynrad_stream_t stream) {
+  if (status_out == nullptr) return DYNRAD_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  int32_t v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_status, sizeof(v), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return DYNRAD_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DYNRAD_ERR_CUDA;
+  *status_out = v;
+  if (clear) {
+    const int32_t zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return DYNRAD_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DYNRAD_ERR_CUDA;
+  }
+  return DYNRAD_OK;
+}
+
+int dynrad_build_candidates(const dynrad_geom* geom, int32_t* cand_row_ptr, int32_t* cand_col,
+                            int64_t cand_cap, int32_t* forced_lo, int32_t* forced_hi,
+                            int64_t* nnz_out, int64_t* max_row_out, dynrad_stream_t stream) {
+  GeomDev g;
+  int rc = check_geom(geom, &g);
+  if (rc != DYNRAD_OK) return rc;
+  if (cand_row_ptr == nullptr || forced_lo == nullptr || forced_hi == nullptr) return DYNRAD_ERR_INVALID_ARG;
+  if (cand_col == nullptr && nnz_out == nullptr) return DYNRAD_ERR_INVALID_ARG;
+  if (cand_col != nullptr && cand_cap < 0) return DYNRAD_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  const size_t tab = static_cast<size_t>(g.frames) * 5 + 16;
+  cand_count_kernel<<<g.nb, kCandThreads, tab, st>>>(g, cand_row_ptr, forced_lo, forced_hi);
+  if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  scan_small_kernel<<<1, 1024, 0, st>>>(cand_row_ptr, g.nb);
+  if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  if (cand_col != nullptr) {
+    cand_fill_kernel<<<g.nb, kCandThreads, tab, st>>>(g, cand_row_ptr, cand_col, cand_cap);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  }
+  if (nnz_out != nullptr || max_row_out != nullptr) {
+    std::vector<int32_t> h(static_cast<size_t>(g.nb) + 1);
+    if (cudaMemcpyAsync(h.data(), cand_row_ptr, h.size() * 4, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+      return DYNRAD_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DYNRAD_ERR_CUDA;
+    int64_t mx = 0;
+    for (int i = 0; i < g.nb; ++i) mx = std::max<int64_t>(mx, h[i + 1] - h[i]);
+    if (nnz_out != nullptr) *nnz_out = h[g.nb];
+    if (max_row_out != nullptr) *max_row_out = mx;
+    if (cand_col != nullptr && h[g.nb] > cand_cap) return DYNRAD_ERR_CAPACITY;
+  }
+  return DYNRAD_OK;
+}
+
+size_t dynrad_select_workspace_bytes(int32_t B, int32_t H, int32_t N, int32_t D, const dynrad_geom* geom,
+                                     int64_t cand_nnz) {
+  GeomDev g;
+  if (check_geom(geom, &g) != DYNRAD_OK || B < 1 || H < 1 || N != g.n || (D != 64 && D != 128) ||
+      cand_nnz < 0)
+    return 0;
+  return select_layout(static_cast<int64_t>(B) * H, g.nb, D, cand_nnz).total;
+}
+
+int dynrad_select_blocks(const void* q, const void* k, int32_t B, int32_t H, int32_t N, int32_t D,
+                         const dynrad_geom* geom, const int32_t* cand_row_ptr, const int32_t* cand_col,
+                         int64_t cand_nnz, int64_t cand_max_row, const int32_t* forced_lo,
+                         const int32_t* forced_hi,
+                         int32_t mode, double rho_or_tau, int32_t* row_ptr, int32_t* col_idx,
+                         int64_t col_cap, float* scores_out, void* workspace, size_t workspace_bytes,
+                         dynrad_stream_t stream) {
+  GeomDev g;
+  int rc = check_geom(geom, &g);
+  if (rc != DYNRAD_OK) return rc;
+  if (q == nullptr || k == nullptr || cand_row_ptr == nullptr || cand_col == nullptr ||
+      forced_lo == nullptr || forced_hi == nullptr || row_ptr == nullptr || col_idx == nullptr ||
+      workspace == nullptr)
+    return DYNRAD_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N != g.n || cand_nnz < 1 || col_cap < 0 || cand_max_row < 0)
+    return DYNRAD_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return DYNRAD_ERR_UNSUPPORTED;
+  if (mode != DYNRAD_STATIC_RATIO && mode != DYNRAD_DYNAMIC_THRESHOLD) return DYNRAD_ERR_INVALID_ARG;
+  if (!(rho_or_tau > 0.0 && rho_or_tau <= 1.0)) return DYNRAD_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return DYNRAD_ERR_INVALID_ARG;
+  if (g.nb > kMaxBlocks) return DYNRAD_ERR_UNSUPPORTED;
+  const int64_t bh = static_cast<int64_t>(B) * H;
+  if (bh > 65535) return DYNRAD_ERR_UNSUPPORTED;
+  if (bh * cand_nnz > INT32_MAX) return DYNRAD_ERR_UNSUPPORTED;
+  const SelectWorkspace w = select_layout(bh, g.nb, D, cand_nnz);
+  if (workspace_bytes < w.total) return DYNRAD_ERR_CAPACITY;
+  cudaStream_t st = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* qbar = reinterpret_cast<float*>(ws + w.qbar);
+  float* kbar = reinterpret_cast<float*>(ws + w.kbar);
+  int32_t* kept = reinterpret_cast<int32_t*>(ws + w.kept);
+  int64_t* partial = reinterpret_cast<int64_t*>(ws + w.partial);
+  const int64_t rows = bh * g.nb;
+
+  // pooling
+  {
+    const int64_t warps = 2 * rows;
+    const int64_t blocks = (warps * 32 + kPoolThreads - 1) / kPoolThreads;
+    if (D == 128)
+      pool_kernel<128><<<static_cast<unsigned>(blocks), kPoolThreads, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), qbar, kbar, N, g.block,
+          g.nb, rows);
+    else
+      pool_kernel<64><<<static_cast<unsigned>(blocks), kPoolThreads, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), qbar, kbar, N, g.block,
+          g.nb, rows);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  }
+  // scoring + selection; shared memory sized for the longest candidate row
+  {
+    SelectParams sp;
+    sp.qbar = qbar;
+    sp.kbar = kbar;
+    sp.cand_row_ptr = cand_row_ptr;
+    sp.cand_col = cand_col;
+    sp.forced_lo = forced_lo;
+    sp.forced_hi = forced_hi;
+    sp.counts = row_ptr;
+    sp.kept_tmp = kept;
+    sp.scores_out = scores_out;
+    sp.cand_nnz = cand_nnz;
+    sp.nb = g.nb;
+    sp.max_row = (cand_max_row > 0 && cand_max_row < g.nb) ? static_cast<int>(cand_max_row) : g.nb;
+    sp.mode = mode;
+    sp.value = rho_or_tau;
+    sp.scale = 1.0f / std::sqrt(static_cast<float>(D));
+    const size_t smem = sel_smem_bytes(D, g.nb, sp.max_row);
+    if (smem > 227 * 1024) return DYNRAD_ERR_UNSUPPORTED;
+    dim3 grid((g.nb + kSelRows - 1) / kSelRows, static_cast<unsigned>(bh));
+    if (D == 128) {
+      if (cudaFuncSetAttribute(score_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem)) != cudaSuccess)
+        return DYNRAD_ERR_CUDA;
+      score_select_kernel<128><<<grid, kSelThreads, smem, st>>>(sp);
+    } else {
+      if (cudaFuncSetAttribute(score_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem)) != cudaSuccess)
+        return DYNRAD_ERR_CUDA;
+      score_select_kernel<64><<<grid, kSelThreads, smem, st>>>(sp);
+    }
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  }
+  // counts -> offsets, compaction
+  {
+    const int64_t tiles = (rows + 1 + kScanTile - 1) / kScanTile;
+    scan_partial_kernel<<<static_cast<unsigned>(tiles), kScanThreads, 0, st>>>(row_ptr, rows, partial);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+    CompactParams cp;
+    cp.row_ptr = row_ptr;
+    cp.partial = partial;
+    cp.rows = rows;
+    cp.nb = g.nb;
+    cp.cand_row_ptr = cand_row_ptr;
+    cp.kept_tmp = kept;
+    cp.cand_nnz = cand_nnz;
+    cp.col_idx = col_idx;
+    cp.col_cap = col_cap;
+    scan_apply_kernel<<<static_cast<unsigned>(tiles), kScanThreads, 0, st>>>(cp);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  }
+  return DYNRAD_OK;
+}
+
+int dynrad_sparse_attn(const void* q, const void* k, const void* v, int32_t B, int32_t H, int32_t N,
+                       int32_t D, int32_t block, const int32_t* row_ptr, const int32_t* col_idx, float scale,
+                       void* o, float* lse, dynrad_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || row_ptr == nullptr || col_idx == nullptr ||
+      o == nullptr || lse == nullptr)
+    return DYNRAD_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1) return DYNRAD_ERR_INVALID_ARG;
+  if (!(scale >= 0.0f) || !std::isfinite(scale)) return DYNRAD_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return DYNRAD_ERR_UNSUPPORTED;
+  if (block != 32 && block != 64 && block != 128) return DYNRAD_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return DYNRAD_ERR_INVALID_ARG;
+  const int64_t bh = static_cast<int64_t>(B) * H;
+  if (bh > 65535) return DYNRAD_ERR_UNSUPPORTED;
+  const int64_t nb = (static_cast<int64_t>(N) + block - 1) / block;
+  if (static_cast<int64_t>(N) * D * 2 >= (int64_t(1) << 40)) return DYNRAD_ERR_UNSUPPORTED;
+  if ((nb + 128 / block - 1) / (128 / block) > INT32_MAX) return DYNRAD_ERR_UNSUPPORTED;
+  const float sc = scale == 0.0f ? 1.0f / std::sqrt(static_cast<float>(D)) : scale;
+  cudaStream_t st = as_stream(stream);
+  const int bhi = static_cast<int>(bh);
+  if (D == 128) {
+    if (block == 32) return launch_attn<128, 32>(q, k, v, bhi, N, row_ptr, col_idx, sc, o, lse, st);
+    if (block == 64) return launch_attn<128, 64>(q, k, v, bhi, N, row_ptr, col_idx, sc, o, lse, st);
+    return launch_attn<128, 128>(q, k, v, bhi, N, row_ptr, col_idx, sc, o, lse, st);
+  }
+  if (block == 32) return launch_attn<64, 32>(q, k, v, bhi, N, row_ptr, col_idx, sc, o, lse, st);
+  if (block == 64) return launch_attn<64, 64>(q, k, v, bhi, N, row_ptr, col_idx, sc, o, lse, st);
+  return launch_attn<64, 128>(q, k, v, bhi, N, row_ptr, col_idx, sc, o, lse, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,194 @@
+/*
+ * dynrad.h -- C ABI of the DynamicRad block-sparse attention hot path on
+ * NVIDIA B200 (sm_100a).
+ *
+ * Source of the method: "DynamicRad: Content-Adaptive Sparse Attention for
+ * Long Video Diffusion" (arXiv 2604.20470).  Three stages:
+ *
+ *   1. dynrad_build_candidates -- the radial candidate block set of Sec. 3.1
+ *      (Eqs. 1-7, "Density control within blocks"; Algorithm 1 lines 4-14, 23).
+ *   2. dynrad_select_blocks    -- per query block, mean-pooled block scores
+ *      (the 1/sqrt(d) logit scale of Eq. 9) and one of the two selection modes
+ *      of Sec. 3.2: static-ratio (top rho fraction, k rule of Eq. 8) or
+ *      dynamic-threshold (smallest prefix whose softmax block mass reaches
+ *      tau).  Output: CSR block indices.
+ *   3. dynrad_sparse_attn      -- block-sparse softmax attention over the kept
+ *      blocks, Eqs. 12-13 with epsilon -> 0, returning O and the log-sum-exp.
+ *
+ * Conventions shared by every call
+ *   - Pointers named q, k, v, o, lse, *_row_ptr, *_col*, forced_*, scores_out,
+ *     workspace are DEVICE pointers owned by the caller.  Geometry structs and
+ *     *_out scalars are HOST pointers.
+ *   - Q, K, V, O are bf16, layout [B, H, N, D] contiguous (D fastest), base
+ *     address 16-byte aligned.  LSE is fp32 [B, H, N].
+ *   - Token t of a head sits at frame t / (height*width), in-frame index
+ *     t % (height*width) (row-major h * width + w).  Blocks are contiguous runs
+ *     of `block` tokens; the last block may be partial (padded keys are never
+ *     attended, padded query rows are never written).  Nb = ceil(N / block).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) unless stated.  The library allocates no memory and frees none of
+ *     the caller's.
+ *   - Every call returns a dynrad_status.  Argument errors are found on the
+ *     host before any launch.  Errors found by a kernel (capacity exceeded, a
+ *     bounded wait that ran out) are recorded in a device status word read by
+ *     dynrad_device_status().
+ */
+#ifndef DYNRAD_H
+#define DYNRAD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *dynrad_stream_t; /* same type as cudaStream_t */
+
+typedef enum dynrad_status {
+  DYNRAD_OK = 0,
+  DYNRAD_ERR_INVALID_ARG = 1, /* null pointer, bad size, parameter out of range */
+  DYNRAD_ERR_UNSUPPORTED = 2, /* head dim / block size / size limit not built */
+  DYNRAD_ERR_CAPACITY = 3,    /* an output or workspace buffer is too small */
+  DYNRAD_ERR_CUDA = 4,        /* a CUDA runtime or launch error */
+  DYNRAD_ERR_DEVICE = 5       /* a kernel-side check or bounded wait failed */
+} dynrad_status;
+
+typedef enum dynrad_mode {
+  DYNRAD_STATIC_RATIO = 0,     /* Sec. 3.2 "Static-ratio mode" (block-pooled top rho) */
+  DYNRAD_DYNAMIC_THRESHOLD = 1 /* Sec. 3.2 "Dynamic-threshold mode" (softmax mass tau) */
+} dynrad_mode;
+
+/* Latent grid and radial parameters (Sec. 3.1; parameter list of Table 4). */
+typedef struct dynrad_geom {
+  int32_t frames;  /* N_f */
+  int32_t height;  /* latent grid rows per frame */
+  int32_t width;   /* latent grid columns per frame; N_t = height * width */
+  int32_t block;   /* B_s, tokens per block: 32, 64 or 128 for attention; any >= 1 here */
+  double gamma;    /* decay factor of Eq. 2, > 0 */
+  double lambda;   /* long-range factor of Eq. 4, > 0 */
+  double theta_c;  /* column density threshold, [0, 1] (0 = any linked query) */
+  double theta_m;  /* block activation threshold, [0, 1] (0 = any active column) */
+  double eps;      /* epsilon of Eq. 5, >= 0 (1e-6 in this library's workloads) */
+  int32_t force_t; /* frame distances <= force_t (0 or 1) are always kept */
+} dynrad_geom;
+
+/* Number of blocks Nb = ceil(frames*height*width / block); 0 on a bad geometry. */
+int64_t dynrad_num_blocks(const dynrad_geom *geom);
+
+/*
+ * Stage 1: radial candidate set (Eqs. 1-7 and the (theta_c, theta_m) block
+ * aggregation of Sec. 3.1), plus each row's always-kept range.
+ *
+ * For query block I the candidates are the blocks J for which the token pairs
+ * (q in I, k in J) that lie in P(frame(q), frame(k)) of Eq. 7 -- the frame pair
+ * retained by the split rule of Eq. 6 and |u - v| <= w of Eq. 3 -- pass the
+ * aggregation: more than theta_c * n_I linked query tokens makes a key token
+ * active, more than theta_m * n_J active key tokens makes J a candidate.  To
+ * that set is added the forced range [forced_lo[I], forced_hi[I]]: the blocks
+ * holding a token whose frame is within force_t of a frame of I (over frame
+ * pairs the split rule retains).  It always contains I itself.
+ *
+ *   cand_row_ptr  device int32 [Nb + 1]  CSR row offsets (written in both modes)
+ *   cand_col      device int32 [cand_cap] ascending block indices per row, or
+ *                 NULL for the size query
+ *   forced_lo/hi  device int32 [Nb] each (written in both modes)
+ *   nnz_out       host; if non-NULL receives the total candidate count and the
+ *                 call SYNCHRONIZES the stream.  Required when cand_col == NULL.
+ *   max_row_out   host, optional; receives the longest row (same sync).
+ * Size query: cand_col == NULL.  Fill: cand_col != NULL; if the total exceeds
+ * cand_cap, nothing past cand_cap is written and the device status becomes
+ * DYNRAD_ERR_CAPACITY (or the call returns it when nnz_out is given).
+ * The candidate set depends only on the geometry, not on Q/K: it can be built
+ * once and reused, as the paper caches static masks (App. D).
+ */
+int dynrad_build_candidates(const dynrad_geom *geom, int32_t *cand_row_ptr,
+                            int32_t *cand_col, int64_t cand_cap,
+                            int32_t *forced_lo, int32_t *forced_hi,
+                            int64_t *nnz_out, int64_t *max_row_out,
+                            dynrad_stream_t stream);
+
+/* Workspace bytes dynrad_select_blocks needs (pooled means + kept lists). */
+size_t dynrad_select_workspace_bytes(int32_t B, int32_t H, int32_t N, int32_t D,
+                                     const dynrad_geom *geom, int64_t cand_nnz);
+
+/*
+ * Stage 2: block pooling, scoring and selection (Sec. 3.2, Algorithm 1 lines
+ * 15-22, in the block-pooled form).
+ *
+ * For every (b, h) and query block I: qbar_I, kbar_J = fp32 means of Q and K
+ * over the valid tokens of each block; s_IJ = qbar_I . kbar_J * (1/sqrt(D))
+ * in fp32 for every candidate J.  F_I = the forced range, N_I = the other
+ * candidates, ranked by (s descending, J ascending).
+ *   mode DYNRAD_STATIC_RATIO, value rho in (0, 1]: keep F_I and the first
+ *     k = max(1, floor(rho * |N_I| + 1e-9)) of N_I (k = 0 if N_I is empty).
+ *   mode DYNRAD_DYNAMIC_THRESHOLD, value tau in (0, 1]: with
+ *     e_J = exp(s_J - max s) (fp64 from the fp32 scores) and Z their sum over
+ *     the candidates, keep F_I and the shortest prefix of N_I such that
+ *     sum_{F_I} e + sum_{prefix} e >= tau * Z.  tau = 1 keeps every candidate.
+ * Kept blocks are written ascending.
+ *
+ *   q, k          device bf16 [B, H, N, D]; N must equal frames*height*width
+ *   D             64 or 128
+ *   cand_*, forced_*   stage-1 output for the same geometry; cand_nnz its total
+ *   cand_max_row  longest candidate row (stage 1's max_row_out), or 0 for the
+ *                 bound Nb; it sizes shared memory.  A row longer than this is
+ *                 an error (device status DYNRAD_ERR_CAPACITY, row left empty)
+ *   row_ptr       device int32 [B*H*Nb + 1]; row (b*H + h)*Nb + I
+ *   col_idx       device int32 [col_cap]; col_cap >= B*H*cand_nnz always suffices
+ *   scores_out    device fp32 [B*H*cand_nnz] or NULL: the fp32 scores in
+ *                 candidate order, row (b, h, I) at (b*H+h)*cand_nnz + cand_row_ptr[I]
+ *   workspace     device, >= dynrad_select_workspace_bytes(...) bytes, 256-byte aligned
+ * If the kept total exceeds col_cap the device status becomes DYNRAD_ERR_CAPACITY
+ * and col_idx is left partial.
+ */
+int dynrad_select_blocks(const void *q, const void *k, int32_t B, int32_t H,
+                         int32_t N, int32_t D, const dynrad_geom *geom,
+                         const int32_t *cand_row_ptr, const int32_t *cand_col,
+                         int64_t cand_nnz, int64_t cand_max_row,
+                         const int32_t *forced_lo,
+                         const int32_t *forced_hi, int32_t mode,
+                         double rho_or_tau, int32_t *row_ptr, int32_t *col_idx,
+                         int64_t col_cap, float *scores_out, void *workspace,
+                         size_t workspace_bytes, dynrad_stream_t stream);
+
+/*
+ * Stage 3: block-sparse attention forward (Eq. 13 with epsilon -> 0).
+ *
+ * For every (b, h) and query token q of block I:
+ *   o_q   = sum_{J in kept(I)} sum_{valid k in J} softmax_k(scale * q.k) v_k
+ *   lse_q = ln sum_{same keys} exp(scale * q.k)
+ * Tensor cores (tcgen05, bf16 operands, fp32 accumulation in TMEM) compute
+ * Q K^T and P V; the softmax runs in fp32.  Rows with no kept block get
+ * o = 0 and lse = -inf.
+ *
+ *   q, k, v       device bf16 [B, H, N, D], D = 64 or 128
+ *   block         32, 64 or 128 (the CSR's block size)
+ *   row_ptr       device int32 [B*H*Nb + 1]; col_idx device int32, strictly
+ *                 ascending block indices in [0, Nb) per row (entries outside
+ *                 the range are skipped and flagged in the device status)
+ *   scale         logit scale; 0 means 1/sqrt(D)
+ *   o             device bf16 [B, H, N, D]; lse device fp32 [B, H, N]
+ */
+int dynrad_sparse_attn(const void *q, const void *k, const void *v, int32_t B,
+                       int32_t H, int32_t N, int32_t D, int32_t block,
+                       const int32_t *row_ptr, const int32_t *col_idx,
+                       float scale, void *o, float *lse,
+                       dynrad_stream_t stream);
+
+/*
+ * Reads the device status word (the first error a kernel recorded since the
+ * last clear) into *status_out; clears it when clear != 0.  SYNCHRONIZES the
+ * stream.  Returns DYNRAD_ERR_CUDA if the stream itself reports an error.
+ */
+int dynrad_device_status(int32_t *status_out, int32_t clear,
+                         dynrad_stream_t stream);
+
+/* Static string for a status code ("ok", "invalid argument", ...). */
+const char *dynrad_status_string(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DYNRAD_H */
