@@ -13,7 +13,7 @@ ctypes with the same names:
 lazily so that the workload generator can be used without a GPU.
 """
 
-_ABI_NAMES = ("dynrad_num_blocks", "dynrad_build_candidates", "dynrad_select_blocks",
+_ABI_NAMES = ("dynrad_num_blocks", "dynrad_build_candidates", "dynrad_build_candidates_into", "dynrad_select_blocks",
               "dynrad_sparse_attn", "dynrad_device_status", "dynrad_select_workspace_bytes",
               "SelectBuffers", "DynradError", "make_geom", "lib")
 

@@ -161,6 +161,16 @@ def dynrad_build_candidates(geom, device=None, stream=None) -> dict:
             "nnz": nnz.value, "max_row": mx.value, "nb": nb}
 
 
+def dynrad_build_candidates_into(geom, cand: dict, stream=None) -> None:
+    """Stage 1 into existing buffers (from dynrad_build_candidates): the fill
+    call only, asynchronous, no host synchronization."""
+    L = lib()
+    cg = make_geom(geom)
+    _check(L.dynrad_build_candidates(ctypes.byref(cg), _ptr(cand["row_ptr"]), _ptr(cand["col"]),
+                                     cand["col"].numel(), _ptr(cand["forced_lo"]), _ptr(cand["forced_hi"]),
+                                     None, None, _stream(stream)), "dynrad_build_candidates")
+
+
 def dynrad_select_workspace_bytes(B, H, N, D, geom, cand_nnz) -> int:
     return int(lib().dynrad_select_workspace_bytes(B, H, N, D, ctypes.byref(make_geom(geom)), cand_nnz))
 
