@@ -42,7 +42,7 @@ from block_sparse_attention_candidate_b200.workloads import (  # noqa: E402
 METRIC = ("sparse-attn effective TFLOPS (kept blocks) at Wan-14B 720p, whole path "
           "(candidates + selection + attention) per step")
 UNIT = "TFLOP/s"
-KERNELS_PER_RUN = 8   # 3 candidate kernels, 4 selection kernels, 1 attention kernel
+KERNELS_PER_RUN = 9   # 3 candidate kernels, 5 selection kernels, 1 attention kernel
 
 
 # ----------------------------------------------------------------------------
@@ -67,6 +67,17 @@ def kept_flops(row_ptr: np.ndarray, col: np.ndarray, n: int, block: int, bh: int
     kept_tok = np.where(counts > 0, kept_tok, 0)
     rows_n = np.tile(nvalid, bh)
     return float(4.0 * d * np.sum(rows_n.astype(np.float64) * kept_tok))
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank timing over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized() or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def load_peaks():
@@ -336,11 +347,7 @@ def main():
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    total_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
     ms_step = total_ms / args.steps
     st = abi.dynrad_device_status(clear=True)
     if st != 0:
@@ -427,11 +434,7 @@ def main():
             e2e_step()
         a1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = a0.elapsed_time(a1)
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
+        e2e_ms = max_over_ranks(a0.elapsed_time(a1), dev)
         e2e = {"value": world * flops_step * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms / args.steps}

@@ -77,7 +77,7 @@ SelectWorkspace select_layout(int64_t bh, int64_t nb, int64_t d, int64_t cand_nn
   const int64_t tiles = (rows + 1 + kScanTile - 1) / kScanTile;
   w.qbar = 0;
   w.kbar = align256(w.qbar + static_cast<size_t>(rows * d) * 4);
-  w.kept = align256(w.kbar + static_cast<size_t>(rows * d) * 4);
+  w.kept = align256(w.kbar + static_cast<size_t>(bh * d * padded_blocks(static_cast<int>(nb))) * 4);
   w.partial = align256(w.kept + static_cast<size_t>(bh * cand_nnz) * 4);
   w.total = align256(w.partial + static_cast<size_t>(tiles) * 8);
   return w;
@@ -119,8 +119,10 @@ int launch_attn(const void* q, const void* k, const void* v, int BH, int N, cons
                 const int32_t* col_idx, float scale, void* o, float* lse, cudaStream_t st) {
   using C = AttnCfg<D, BS>;
   CUtensorMap mq, mk, mv;
-  if (!encode_map(&mq, q, D, N, BH, 128) || !encode_map(&mk, k, D, N, BH, BS) ||
-      !encode_map(&mv, v, D, N, BH, BS))
+  // K / V boxes are one key step (C::kKW rows), the unit the kernel's ring
+  // slots and transaction counts are sized for
+  if (!encode_map(&mq, q, D, N, BH, C::kM) || !encode_map(&mk, k, D, N, BH, C::kKW) ||
+      !encode_map(&mv, v, D, N, BH, C::kKW))
     return DYNRAD_ERR_CUDA;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
@@ -256,30 +258,18 @@ int dynrad_select_blocks(const void* q, const void* k, int32_t B, int32_t H, int
   cudaStream_t st = as_stream(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* qbar = reinterpret_cast<float*>(ws + w.qbar);
-  float* kbar = reinterpret_cast<float*>(ws + w.kbar);
+  float* kbarT = reinterpret_cast<float*>(ws + w.kbar);
   int32_t* kept = reinterpret_cast<int32_t*>(ws + w.kept);
   int64_t* partial = reinterpret_cast<int64_t*>(ws + w.partial);
   const int64_t rows = bh * g.nb;
 
-  // pooling
+  // pooling, then scoring + selection
   {
-    const int64_t warps = 2 * rows;
-    const int64_t blocks = (warps * 32 + kPoolThreads - 1) / kPoolThreads;
-    if (D == 128)
-      pool_kernel<128><<<static_cast<unsigned>(blocks), kPoolThreads, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), qbar, kbar, N, g.block,
-          g.nb, rows);
-    else
-      pool_kernel<64><<<static_cast<unsigned>(blocks), kPoolThreads, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), qbar, kbar, N, g.block,
-          g.nb, rows);
-    if ((rc = launch_status()) != DYNRAD_OK) return rc;
-  }
-  // scoring + selection; shared memory sized for the longest candidate row
-  {
-    SelectParams sp;
+    Stage2Params sp;
+    sp.q = static_cast<const __nv_bfloat16*>(q);
+    sp.k = static_cast<const __nv_bfloat16*>(k);
     sp.qbar = qbar;
-    sp.kbar = kbar;
+    sp.kbarT = kbarT;
     sp.cand_row_ptr = cand_row_ptr;
     sp.cand_col = cand_col;
     sp.forced_lo = forced_lo;
@@ -288,25 +278,33 @@ int dynrad_select_blocks(const void* q, const void* k, int32_t B, int32_t H, int
     sp.kept_tmp = kept;
     sp.scores_out = scores_out;
     sp.cand_nnz = cand_nnz;
+    sp.N = N;
+    sp.block = g.block;
     sp.nb = g.nb;
+    sp.nbp = padded_blocks(g.nb);
     sp.max_row = (cand_max_row > 0 && cand_max_row < g.nb) ? static_cast<int>(cand_max_row) : g.nb;
     sp.mode = mode;
     sp.value = rho_or_tau;
     sp.scale = 1.0f / std::sqrt(static_cast<float>(D));
-    const size_t smem = sel_smem_bytes(D, g.nb, sp.max_row);
+    const int nq = (g.nb + kSelRows - 1) / kSelRows;
+    const dim3 pgrid(2 * nq, static_cast<unsigned>(bh));
+    if (D == 128)
+      pool_kernel<128><<<pgrid, kS2Threads, 0, st>>>(sp);
+    else
+      pool_kernel<64><<<pgrid, kS2Threads, 0, st>>>(sp);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+    const size_t smem = s2_smem_bytes(D, g.nb, sp.max_row);
     if (smem > 227 * 1024) return DYNRAD_ERR_UNSUPPORTED;
-    dim3 grid((g.nb + kSelRows - 1) / kSelRows, static_cast<unsigned>(bh));
-    if (D == 128) {
-      if (cudaFuncSetAttribute(score_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem)) != cudaSuccess)
-        return DYNRAD_ERR_CUDA;
-      score_select_kernel<128><<<grid, kSelThreads, smem, st>>>(sp);
-    } else {
-      if (cudaFuncSetAttribute(score_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem)) != cudaSuccess)
-        return DYNRAD_ERR_CUDA;
-      score_select_kernel<64><<<grid, kSelThreads, smem, st>>>(sp);
-    }
+    const void* kern = D == 128 ? reinterpret_cast<const void*>(select_kernel<128>)
+                                : reinterpret_cast<const void*>(select_kernel<64>);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+        cudaSuccess)
+      return DYNRAD_ERR_CUDA;
+    const dim3 sgrid(nq, static_cast<unsigned>(bh));
+    if (D == 128)
+      select_kernel<128><<<sgrid, kS2Threads, smem, st>>>(sp);
+    else
+      select_kernel<64><<<sgrid, kS2Threads, smem, st>>>(sp);
     if ((rc = launch_status()) != DYNRAD_OK) return rc;
   }
   // counts -> offsets, compaction
@@ -325,6 +323,9 @@ int dynrad_select_blocks(const void* q, const void* k, int32_t B, int32_t H, int
     cp.col_idx = col_idx;
     cp.col_cap = col_cap;
     scan_apply_kernel<<<static_cast<unsigned>(tiles), kScanThreads, 0, st>>>(cp);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+    const int64_t cblocks = (rows * 32 + kCompactThreads - 1) / kCompactThreads;
+    compact_kernel<<<static_cast<unsigned>(cblocks), kCompactThreads, 0, st>>>(cp);
     if ((rc = launch_status()) != DYNRAD_OK) return rc;
   }
   return DYNRAD_OK;

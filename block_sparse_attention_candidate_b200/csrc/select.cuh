@@ -1,17 +1,18 @@
 // Stage 2: block pooling, block proxy scores and the two selection modes
 // (DynamicRad, Sec. 3.2 and Algorithm 1 lines 15-22, in block-pooled form).
 //
-//   pool_kernel          qbar, kbar = fp32 means of Q, K over each block's valid
-//                        tokens.  HBM-bound: one warp streams one 64x128 bf16
-//                        block with 16-byte loads, shuffle-reduces, writes 512 B.
-//   score_select_kernel  one CTA = 8 consecutive query blocks of one head.  The
-//                        union of their candidate lists is scored once per key
-//                        block (register blocking over the 8 rows: each kbar row
-//                        read from L2 feeds 8 dot products), then each warp
-//                        selects for its row by a 4-pass radix descent over the
-//                        order-preserving 32-bit score keys.
-//   scan_*_kernel        kept counts -> CSR row offsets, and compaction of the
-//                        per-row kept lists into col_idx.
+// Two launches:
+//
+//   pool_kernel    one CTA per (tensor, head, 8 consecutive blocks): each warp
+//                  streams one block (B_s x D bf16, 16-byte loads), shuffle-reduces,
+//                  and writes the fp32 mean -- qbar row-major [BH, Nb, D], kbar
+//                  transposed [BH, D, NbP] through a shared-memory transpose so the
+//                  score loads below are coalesced.  HBM-bound.
+//   select_kernel  one CTA per (head, 8 consecutive query blocks): the union of the
+//                  8 candidate lists is scored once per key block (each kbar value
+//                  read feeds 8 dot products, packed f32x2 FMAs), then each warp
+//                  selects for its row by a 4-pass radix descent over
+//                  order-preserving score keys.
 //
 // Ranking: (score descending, block index ascending).  Scores compare as
 // numbers: -0 is folded into +0 before the key is formed.  Static mode weighs
@@ -20,15 +21,15 @@
 // fixed point, so every mass sum is an exact, order-independent integer sum;
 // it looks for the shortest ranking prefix whose weight, added to the forced
 // weight, reaches tau * Z.
+//
+//   scan_*_kernel        kept counts -> CSR row offsets.
+//   compact_kernel       per-row kept lists -> col_idx (one warp per row).
 #pragma once
 
 #include "common.cuh"
 
 namespace dynrad {
 
-// ---------------------------------------------------------------------------
-// pooling
-// ---------------------------------------------------------------------------
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -46,79 +47,34 @@ __device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4& v) {
   }
 }
 
-constexpr int kPoolThreads = 256;
-
-// One warp per (tensor in {Q, K}, b*H + h, block).
-template <int D>
-__global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16* __restrict__ q,
-                                                            const __nv_bfloat16* __restrict__ k,
-                                                            float* __restrict__ qbar,
-                                                            float* __restrict__ kbar, int N,
-                                                            int block, int nb, int64_t rows) {
-  constexpr int LPR = D / 8;      // lanes per token row (8 bf16 = 16 B each)
-  constexpr int RPI = 32 / LPR;   // token rows per warp iteration
-  constexpr int UNROLL = 8;
-  const int lane = threadIdx.x & 31;
-  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * kPoolThreads + threadIdx.x) >> 5;
-  if (wid >= 2 * rows) return;
-  const bool is_k = wid >= rows;
-  const int64_t r = is_k ? wid - rows : wid;
-  const int64_t bh = r / nb;
-  const int blk = static_cast<int>(r - bh * nb);
-  const int t0 = blk * block;
-  const int nvalid = min(block, N - t0);
-  const __nv_bfloat16* src = (is_k ? k : q) + (static_cast<size_t>(bh) * N + t0) * D;
-  const int sub = lane / LPR;
-  const int c8 = (lane % LPR) * 8;
-  float acc[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  int t = sub;
-  for (; t + (UNROLL - 1) * RPI < nvalid; t += UNROLL * RPI) {
-    uint4 v[UNROLL];
-#pragma unroll
-    for (int u = 0; u < UNROLL; ++u) v[u] = ldg_stream(src + static_cast<size_t>(t + u * RPI) * D + c8);
-#pragma unroll
-    for (int u = 0; u < UNROLL; ++u) acc_bf16x8(acc, v[u]);
-  }
-  for (; t < nvalid; t += RPI) acc_bf16x8(acc, ldg_stream(src + static_cast<size_t>(t) * D + c8));
-#pragma unroll
-  for (int off = LPR; off < 32; off <<= 1)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
-  if (sub == 0) {
-    float* dst = (is_k ? kbar : qbar) + r * D + c8;
-    const float inv = static_cast<float>(nvalid);
-    float4 a = make_float4(acc[0] / inv, acc[1] / inv, acc[2] / inv, acc[3] / inv);
-    float4 b = make_float4(acc[4] / inv, acc[5] / inv, acc[6] / inv, acc[7] / inv);
-    reinterpret_cast<float4*>(dst)[0] = a;
-    reinterpret_cast<float4*>(dst)[1] = b;
-  }
-}
-
-// ---------------------------------------------------------------------------
-// scoring + selection
-// ---------------------------------------------------------------------------
-constexpr int kSelRows = 8;                 // query blocks per CTA (one warp each)
-constexpr int kSelThreads = kSelRows * 32;
+constexpr int kSelRows = 8;                   // query blocks per score item (one warp each)
+constexpr int kS2Threads = kSelRows * 32;     // 8 warps
 constexpr double kMassScale = 68719476736.0;  // 2^36 fixed-point scale of e_J
 
-struct SelectParams {
-  const float* qbar;
-  const float* kbar;
+// Padded block count of the transposed kbar: rows of 128 bytes.
+__host__ __device__ constexpr int padded_blocks(int nb) { return (nb + 31) & ~31; }
+
+struct Stage2Params {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  float* qbar;              // [BH, nb, D]
+  float* kbarT;             // [BH, D, nbp]
   const int32_t* cand_row_ptr;
   const int32_t* cand_col;
   const int32_t* forced_lo;
   const int32_t* forced_hi;
-  int32_t* counts;      // kept count per row (row_ptr before the scan)
-  int32_t* kept_tmp;    // [BH, cand_nnz] kept lists at the candidate offsets
-  float* scores_out;    // nullable
+  int32_t* counts;          // kept count per row (row_ptr before the scan)
+  int32_t* kept_tmp;        // [BH, cand_nnz] kept lists at the candidate offsets
+  float* scores_out;        // nullable
   int64_t cand_nnz;
+  int N;
+  int block;
   int nb;
-  int max_row;          // bound on candidates per row (smem sizing)
+  int nbp;
+  int max_row;              // bound on candidates per row (smem sizing)
   int mode;
-  double value;         // rho or tau
-  float scale;          // 1 / sqrt(D)
+  double value;             // rho or tau
+  float scale;              // 1 / sqrt(D)
 };
 
 // Order-preserving key of a finite float: larger key <=> larger number.
@@ -155,53 +111,114 @@ struct Reach {
   }
 };
 
-// Per-warp selection scratch in shared memory: bins[256] u64, weights[cap] u64,
-// keys[cap] u32, flags[cap] u8, rounded to 16 bytes.
+// Per-warp selection scratch in shared memory: bins 2 x 256 u32, weights[cap]
+// u64, keys[cap] u32, flags[cap] u8, rounded to 16 bytes.
 __host__ __device__ constexpr size_t sel_warp_bytes(int cap) {
   return (2048 + static_cast<size_t>(cap) * 13 + 15) & ~static_cast<size_t>(15);
 }
 
-// Dynamic shared memory of score_select_kernel.
-__host__ __device__ constexpr size_t sel_smem_bytes(int D, int nb, int cap) {
-  return ((static_cast<size_t>(kSelRows) * D * 4 + static_cast<size_t>((nb + 31) / 32) * 4 +
-           static_cast<size_t>((nb + 31) / 32 + 1) * 4 + static_cast<size_t>(nb) * 4 +
-           static_cast<size_t>(kSelRows) * nb * 4 + 15) & ~static_cast<size_t>(15)) +
+// Shared memory of stage2_kernel: [qsT 8*D f32][bitmap][wprefix][ulist nb]
+// [S 8*nb f32 | pool transpose tile 8*D f32][per-warp selection scratch].
+__host__ __device__ constexpr size_t s2_head_bytes(int D, int nb) {
+  return static_cast<size_t>(kSelRows) * D * 4 + static_cast<size_t>((nb + 31) / 32) * 4 +
+         static_cast<size_t>((nb + 31) / 32 + 1) * 4 + static_cast<size_t>(nb) * 4;
+}
+__host__ __device__ constexpr size_t s2_smem_bytes(int D, int nb, int cap) {
+  return ((s2_head_bytes(D, nb) + static_cast<size_t>(kSelRows) * (nb > D ? nb : D) * 4 + 15) &
+          ~static_cast<size_t>(15)) +
          kSelRows * sel_warp_bytes(cap);
 }
 
+// Pool item: warp w pools block 8*grp + w of one (tensor, head).
 template <int D>
-__global__ void __launch_bounds__(kSelThreads) score_select_kernel(SelectParams p) {
-  extern __shared__ __align__(16) uint8_t sel_smem[];
+__device__ __forceinline__ void pool_item(const Stage2Params& p, bool is_k, int bh, int grp,
+                                          float* tile) {
+  constexpr int LPR = D / 8;      // lanes per token row (8 bf16 = 16 B each)
+  constexpr int RPI = 32 / LPR;   // token rows per warp iteration
+  constexpr int UNROLL = 8;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int blk = grp * kSelRows + warp;
+  const int sub = lane / LPR;
+  const int c8 = (lane % LPR) * 8;
+  if (blk < p.nb) {
+    const int t0 = blk * p.block;
+    const int nvalid = min(p.block, p.N - t0);
+    const __nv_bfloat16* src = (is_k ? p.k : p.q) + (static_cast<size_t>(bh) * p.N + t0) * D;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    int t = sub;
+    for (; t + (UNROLL - 1) * RPI < nvalid; t += UNROLL * RPI) {
+      uint4 v[UNROLL];
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) v[u] = ldg_stream(src + static_cast<size_t>(t + u * RPI) * D + c8);
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) acc_bf16x8(acc, v[u]);
+    }
+    for (; t < nvalid; t += RPI) acc_bf16x8(acc, ldg_stream(src + static_cast<size_t>(t) * D + c8));
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+    if (sub == 0) {
+      const float inv = static_cast<float>(nvalid);
+      if (!is_k) {
+        float* dst = p.qbar + (static_cast<int64_t>(bh) * p.nb + blk) * D + c8;
+        reinterpret_cast<float4*>(dst)[0] = make_float4(acc[0] / inv, acc[1] / inv, acc[2] / inv, acc[3] / inv);
+        reinterpret_cast<float4*>(dst)[1] = make_float4(acc[4] / inv, acc[5] / inv, acc[6] / inv, acc[7] / inv);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) tile[warp * D + c8 + i] = acc[i] / inv;
+      }
+    }
+  }
+  if (is_k) {
+    // transpose the 8 blocks' means: kbarT[bh][d][8*grp + w], 32-byte runs
+    __syncthreads();
+    const int nvb = min(kSelRows, p.nb - grp * kSelRows);
+    float* dstT = p.kbarT + static_cast<int64_t>(bh) * D * p.nbp + grp * kSelRows;
+    for (int i = threadIdx.x; i < kSelRows * D; i += kS2Threads) {
+      const int d = i / kSelRows, w = i % kSelRows;
+      if (w < nvb) dstT[static_cast<int64_t>(d) * p.nbp + w] = tile[w * D + d];
+    }
+  }
+}
+
+// Score + select item: rows I0 .. I0+7 of head bh.
+template <int D>
+__device__ __forceinline__ void score_item(const Stage2Params& p, int bh, int I0, uint8_t* sm) {
   const int nb = p.nb;
   const int nwords = (nb + 31) >> 5;
   const int cap = p.max_row;
-  // shared layout
-  float* qs = reinterpret_cast<float*>(sel_smem);                          // [8][D]
-  uint32_t* bitmap = reinterpret_cast<uint32_t*>(qs + kSelRows * D);       // [nwords]
-  int32_t* wprefix = reinterpret_cast<int32_t*>(bitmap + nwords);          // [nwords + 1]
-  int32_t* ulist = wprefix + nwords + 1;                                   // [nb]
-  float* S = reinterpret_cast<float*>(ulist + nb);                         // [8][nb]
-  uintptr_t wp = reinterpret_cast<uintptr_t>(S + static_cast<size_t>(kSelRows) * nb);
+  float* qsT = reinterpret_cast<float*>(sm);                              // [D][8]
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(qsT + kSelRows * D);     // [nwords]
+  int32_t* wprefix = reinterpret_cast<int32_t*>(bitmap + nwords);         // [nwords + 1]
+  int32_t* ulist = wprefix + nwords + 1;                                  // [nb]
+  float* S = reinterpret_cast<float*>(ulist + nb);                        // [8][nb]
+  uintptr_t wp = reinterpret_cast<uintptr_t>(sm) + s2_head_bytes(D, nb) +
+                 static_cast<size_t>(kSelRows) * (nb > D ? nb : D) * 4;
   wp = (wp + 15) & ~static_cast<uintptr_t>(15);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // per-warp arrays: bins[256] u64, wgt[cap] u64, key[cap] u32, flag[cap] u8
   uint8_t* wbase = reinterpret_cast<uint8_t*>(wp) + static_cast<size_t>(warp) * sel_warp_bytes(cap);
-  uint64_t* bins = reinterpret_cast<uint64_t*>(wbase);
-  uint64_t* wgt = bins + 256;
+  uint32_t* bins32 = reinterpret_cast<uint32_t*>(wbase);   // [2][256]: low / high 18-bit sums
+  uint64_t* wgt = reinterpret_cast<uint64_t*>(wbase + 2048);
   uint32_t* key = reinterpret_cast<uint32_t*>(wgt + cap);
   uint8_t* flag = reinterpret_cast<uint8_t*>(key + cap);
 
-  const int64_t bh = blockIdx.y;
-  const int I0 = blockIdx.x * kSelRows;
   const int I = I0 + warp;
   const bool row_ok = I < nb;
+  const bool dynamic = p.mode == DYNRAD_DYNAMIC_THRESHOLD;
+  // Static mode without score export never needs the forced blocks' scores
+  // (they are kept regardless and k counts only the others).
+  const bool skip_forced = !dynamic && p.scores_out == nullptr;
+  const int flo = row_ok ? p.forced_lo[I] : 0, fhi = row_ok ? p.forced_hi[I] : -1;
 
-  // 1. pooled queries of the 8 rows; clear the union bitmap
-  for (int i = threadIdx.x; i < kSelRows * D; i += kSelThreads) {
-    const int r = i / D;
-    qs[i] = (I0 + r < nb) ? p.qbar[(bh * nb + I0 + r) * D + (i % D)] : 0.f;
+  // 1. pooled queries of the 8 rows, transposed; clear the union bitmap
+  for (int i = threadIdx.x; i < kSelRows * D; i += kS2Threads) {
+    const int r = i / D, d = i % D;
+    qsT[d * kSelRows + r] = (I0 + r < nb) ? p.qbar[(static_cast<int64_t>(bh) * nb + I0 + r) * D + d] : 0.f;
   }
-  for (int i = threadIdx.x; i < nwords; i += kSelThreads) bitmap[i] = 0u;
+  for (int i = threadIdx.x; i < nwords; i += kS2Threads) bitmap[i] = 0u;
   __syncthreads();
 
   // 2. union of the 8 candidate lists
@@ -210,15 +227,12 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(SelectParams 
     c_beg = p.cand_row_ptr[I];
     n = p.cand_row_ptr[I + 1] - c_beg;
     if (n > cap || n < 0) {  // longer than the declared bound: the row stays empty
-      if (lane == 0) {
-        record_error(DYNRAD_ERR_CAPACITY);
-        p.counts[bh * nb + I] = 0;
-      }
+      if (lane == 0) record_error(DYNRAD_ERR_CAPACITY);
       n = 0;
     }
     for (int c = lane; c < n; c += 32) {
       const int J = p.cand_col[c_beg + c];
-      atomicOr(&bitmap[J >> 5], 1u << (J & 31));
+      if (!skip_forced || J < flo || J > fhi) atomicOr(&bitmap[J >> 5], 1u << (J & 31));
     }
   }
   __syncthreads();
@@ -230,6 +244,7 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(SelectParams 
       const int w = w0 + lane;
       const int c = w < nwords ? __popc(bitmap[w]) : 0;
       int incl = c;
+#pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += y;
@@ -241,7 +256,7 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(SelectParams 
   }
   __syncthreads();
   const int U = wprefix[nwords];
-  for (int w = threadIdx.x; w < nwords; w += kSelThreads) {
+  for (int w = threadIdx.x; w < nwords; w += kS2Threads) {
     uint32_t bits = bitmap[w];
     int pos = wprefix[w];
     while (bits) {
@@ -252,62 +267,81 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(SelectParams 
   }
   __syncthreads();
 
-  // 4. block scores for every (row, union member); each kbar row feeds 8 rows
-  for (int u = threadIdx.x; u < U; u += kSelThreads) {
-    const float4* kb = reinterpret_cast<const float4*>(p.kbar + (bh * nb + ulist[u]) * D);
-    float acc[kSelRows];
+  // 4. block scores: thread handles union members u and u + 256; each kbar
+  //    value read (coalesced across consecutive members) feeds 8 rows
+  const float* kT = p.kbarT + static_cast<int64_t>(bh) * D * p.nbp;
+  for (int u0 = threadIdx.x; u0 < U; u0 += 2 * kS2Threads) {
+    const int u1 = u0 + kS2Threads;
+    const int J0 = ulist[u0];
+    const int J1 = u1 < U ? ulist[u1] : J0;
+    float2 a0[4], a1[4];
 #pragma unroll
-    for (int r = 0; r < kSelRows; ++r) acc[r] = 0.f;
-#pragma unroll 4
-    for (int d4 = 0; d4 < D / 4; ++d4) {
-      const float4 kv = __ldg(kb + d4);
-#pragma unroll
-      for (int r = 0; r < kSelRows; ++r) {
-        const float4 qv = reinterpret_cast<const float4*>(qs + r * D)[d4];
-        acc[r] = fmaf(qv.x, kv.x, acc[r]);
-        acc[r] = fmaf(qv.y, kv.y, acc[r]);
-        acc[r] = fmaf(qv.z, kv.z, acc[r]);
-        acc[r] = fmaf(qv.w, kv.w, acc[r]);
-      }
+    for (int r = 0; r < 4; ++r) {
+      a0[r] = make_float2(0.f, 0.f);
+      a1[r] = make_float2(0.f, 0.f);
+    }
+#pragma unroll 16
+    for (int d = 0; d < D; ++d) {
+      const float k0 = __ldg(kT + static_cast<int64_t>(d) * p.nbp + J0);
+      const float k1 = __ldg(kT + static_cast<int64_t>(d) * p.nbp + J1);
+      const float4 qa = reinterpret_cast<const float4*>(qsT + d * kSelRows)[0];
+      const float4 qb = reinterpret_cast<const float4*>(qsT + d * kSelRows)[1];
+      const float2 kk0 = make_float2(k0, k0), kk1 = make_float2(k1, k1);
+      const float2 q01 = make_float2(qa.x, qa.y), q23 = make_float2(qa.z, qa.w);
+      const float2 q45 = make_float2(qb.x, qb.y), q67 = make_float2(qb.z, qb.w);
+      a0[0] = __ffma2_rn(q01, kk0, a0[0]);
+      a0[1] = __ffma2_rn(q23, kk0, a0[1]);
+      a0[2] = __ffma2_rn(q45, kk0, a0[2]);
+      a0[3] = __ffma2_rn(q67, kk0, a0[3]);
+      a1[0] = __ffma2_rn(q01, kk1, a1[0]);
+      a1[1] = __ffma2_rn(q23, kk1, a1[1]);
+      a1[2] = __ffma2_rn(q45, kk1, a1[2]);
+      a1[3] = __ffma2_rn(q67, kk1, a1[3]);
     }
 #pragma unroll
-    for (int r = 0; r < kSelRows; ++r) S[r * nb + u] = acc[r] * p.scale;
+    for (int r = 0; r < 4; ++r) {
+      S[(2 * r) * nb + u0] = a0[r].x * p.scale;
+      S[(2 * r + 1) * nb + u0] = a0[r].y * p.scale;
+      if (u1 < U) {
+        S[(2 * r) * nb + u1] = a1[r].x * p.scale;
+        S[(2 * r + 1) * nb + u1] = a1[r].y * p.scale;
+      }
+    }
   }
   __syncthreads();
-  if (!row_ok || n == 0) {
-    if (row_ok && lane == 0) p.counts[bh * nb + I] = 0;
+  if (!row_ok) return;
+  const int64_t bhl = bh;
+  if (n == 0) {
+    if (lane == 0) p.counts[bhl * nb + I] = 0;
     return;
   }
 
   // 5. selection for row I (one warp)
-  const int flo = p.forced_lo[I], fhi = p.forced_hi[I];
   const int32_t* cols = p.cand_col + c_beg;
   const float* Srow = S + warp * nb;
   auto score_of = [&](int J) -> float {
     const int w = J >> 5;
     return Srow[wprefix[w] + __popc(bitmap[w] & ((1u << (J & 31)) - 1u))];
   };
-  const bool dynamic = p.mode == DYNRAD_DYNAMIC_THRESHOLD;
   float smax = -INFINITY;
-  for (int c = lane; c < n; c += 32) smax = fmaxf(smax, score_of(cols[c]));
+  if (dynamic)
+    for (int c = lane; c < n; c += 32) smax = fmaxf(smax, score_of(cols[c]));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, off));
   uint64_t base = 0, ztot = 0;
   int nfree = 0;
   for (int c0 = 0; c0 < n; c0 += 32) {
     const int c = c0 + lane;
-    uint64_t w = 0;
     bool forced = false;
     if (c < n) {
       const int J = cols[c];
-      const float s = score_of(J);
-      if (p.scores_out != nullptr) p.scores_out[bh * p.cand_nnz + c_beg + c] = s;
       forced = J >= flo && J <= fhi;
+      const float s = (forced && skip_forced) ? 0.f : score_of(J);
+      if (p.scores_out != nullptr) p.scores_out[bhl * p.cand_nnz + c_beg + c] = s;
+      uint64_t w = 1;
       if (dynamic) {
         const double e = exp(static_cast<double>(s) - static_cast<double>(smax));
         w = __double2ull_rn(e * kMassScale);
-      } else {
-        w = 1;
       }
       wgt[c] = forced ? 0 : w;
       key[c] = order_key(s);
@@ -340,27 +374,35 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(SelectParams 
 
   uint32_t kstar = 0xFFFFFFFFu;  // cut key; free blocks with key > kstar are kept
   uint64_t above = 0;            // weight of free blocks with key > kstar
-  bool cut_none = !keep_all && reach(0);
+  const bool cut_none = !keep_all && reach(0);
   if (!keep_all && !cut_none) {
     uint32_t prefix = 0, pmask = 0;
     bool found = true;
     for (int pass = 0; pass < 4 && found; ++pass) {
       const int shift = 24 - 8 * pass;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) bins[lane * 8 + i] = 0;
+      for (int i = 0; i < 16; ++i) bins32[lane * 16 + i] = 0u;
       __syncwarp();
+      // weights < 2^36 are split into 18-bit halves; each half's bin sum stays
+      // below 2^32 for rows of up to 2^14 candidates, so native 32-bit shared
+      // atomics give exact sums
       for (int c = lane; c < n; c += 32) {
         if (flag[c]) continue;
         const uint32_t kk = key[c];
-        if ((kk & pmask) == prefix) atomicAdd(reinterpret_cast<unsigned long long*>(&bins[(kk >> shift) & 255u]),
-                                              static_cast<unsigned long long>(wgt[c]));
+        if ((kk & pmask) == prefix) {
+          const uint64_t w = wgt[c];
+          const uint32_t b = (kk >> shift) & 255u;
+          atomicAdd(&bins32[b], static_cast<uint32_t>(w & 0x3FFFFu));
+          if (w >> 18) atomicAdd(&bins32[256 + b], static_cast<uint32_t>(w >> 18));
+        }
       }
       __syncwarp();
       // lane l owns digits 255-8l ... 248-8l (descending)
       uint64_t loc[8], lsum = 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        loc[i] = bins[255 - (lane * 8 + i)];
+        const uint32_t b = 255 - (lane * 8 + i);
+        loc[i] = (static_cast<uint64_t>(bins32[256 + b]) << 18) + bins32[b];
         lsum += loc[i];
       }
       const uint64_t excl = warp_excl_scan_u64(lsum, lane);
@@ -394,31 +436,26 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(SelectParams 
     else keep_all = true;  // target not reachable (rounding at tau ~ 1): keep all
   }
 
-  // 6. mark kept free blocks: key > kstar, and ties at kstar in ascending order
-  //    until the target is reached
+  // 6. mark kept free blocks: key > kstar, and ties at kstar in ascending
+  //    order until the target is reached
   if (!cut_none) {
     uint64_t tie_run = 0;
-    bool done = false;
     for (int c0 = 0; c0 < n; c0 += 32) {
       const int c = c0 + lane;
       bool kept = false;
-      if (c < n && !flag[c]) {
-        const uint32_t kk = key[c];
-        if (keep_all || kk > kstar) kept = true;
-      }
+      if (c < n && !flag[c] && (keep_all || key[c] > kstar)) kept = true;
       const bool tie = !keep_all && c < n && !flag[c] && key[c] == kstar;
       const uint64_t tw = tie ? wgt[c] : 0;
       const uint64_t ex = warp_excl_scan_u64(tw, lane);
-      if (tie && !done && !reach(above + tie_run + ex)) kept = true;
+      if (tie && !reach(above + tie_run + ex)) kept = true;
       tie_run += warp_sum_u64(tw);
-      if (!done && reach(above + tie_run)) done = true;
       if (c < n && kept) flag[c] = 1;
     }
   }
   __syncwarp();
 
   // 7. ordered output of the kept blocks
-  int32_t* dst = p.kept_tmp + bh * p.cand_nnz + c_beg;
+  int32_t* dst = p.kept_tmp + bhl * p.cand_nnz + c_beg;
   int cnt = 0;
   for (int c0 = 0; c0 < n; c0 += 32) {
     const int c = c0 + lane;
@@ -427,7 +464,25 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(SelectParams 
     if (k_) dst[cnt + __popc(bal & ((1u << lane) - 1u))] = cols[c];
     cnt += __popc(bal);
   }
-  if (lane == 0) p.counts[bh * nb + I] = cnt;
+  if (lane == 0) p.counts[bhl * nb + I] = cnt;
+}
+
+// Pool: one CTA per (tensor, head, 8 consecutive blocks); many CTAs per SM keep
+// enough loads in flight to run at HBM bandwidth.
+template <int D>
+__global__ void __launch_bounds__(kS2Threads, 4) pool_kernel(Stage2Params p) {
+  __shared__ __align__(16) float tile[kSelRows * D];
+  const int nq = (p.nb + kSelRows - 1) / kSelRows;
+  const int grp = blockIdx.x % nq;
+  const bool is_k = (blockIdx.x / nq) != 0;
+  pool_item<D>(p, is_k, blockIdx.y, grp, tile);
+}
+
+// Score + select: one CTA per (head, 8 consecutive query blocks).
+template <int D>
+__global__ void __launch_bounds__(kS2Threads, 2) select_kernel(Stage2Params p) {
+  extern __shared__ __align__(16) uint8_t s2_smem[];
+  score_item<D>(p, blockIdx.y, blockIdx.x * kSelRows, s2_smem);
 }
 
 // ---------------------------------------------------------------------------
@@ -527,20 +582,26 @@ __global__ void __launch_bounds__(kScanThreads) scan_apply_kernel(CompactParams 
     if (o > INT32_MAX) record_error(DYNRAD_ERR_CAPACITY);
     p.row_ptr[p.rows] = o > INT32_MAX ? INT32_MAX : static_cast<int32_t>(o);
   }
-  // compaction: warp per row
-  for (int i = warp; i < kScanTile; i += kScanThreads / 32) {
-    const int64_t r = b0 + i;
-    if (r >= p.rows) break;
-    const int64_t bh = r / p.nb;
-    const int I = static_cast<int>(r - bh * p.nb);
-    const int64_t o = offs[i];
-    const int64_t cnt = offs[i + 1] - o;
-    const int32_t* src = p.kept_tmp + bh * p.cand_nnz + p.cand_row_ptr[I];
-    for (int64_t c = lane; c < cnt; c += 32) {
-      const int64_t d = o + c;
-      if (d < p.col_cap) p.col_idx[d] = src[c];
-      else record_error(DYNRAD_ERR_CAPACITY);
-    }
+}
+
+
+// Copies every row's kept list from the candidate-offset scratch to its CSR
+// position: one warp per row.
+constexpr int kCompactThreads = 256;
+
+__global__ void __launch_bounds__(kCompactThreads) compact_kernel(CompactParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (static_cast<int64_t>(blockIdx.x) * kCompactThreads + threadIdx.x) >> 5;
+  if (r >= p.rows) return;
+  const int64_t bh = r / p.nb;
+  const int I = static_cast<int>(r - bh * p.nb);
+  const int64_t o = p.row_ptr[r];
+  const int64_t cnt = static_cast<int64_t>(p.row_ptr[r + 1]) - o;
+  const int32_t* src = p.kept_tmp + bh * p.cand_nnz + p.cand_row_ptr[I];
+  for (int64_t c = lane; c < cnt; c += 32) {
+    const int64_t d = o + c;
+    if (d < p.col_cap) p.col_idx[d] = src[c];
+    else record_error(DYNRAD_ERR_CAPACITY);
   }
 }
 

@@ -109,6 +109,8 @@ def test_workspace_size_formula():
     nnz = 331078
     ws = abi.dynrad_select_workspace_bytes(1, 40, g.n_tokens, 128, g, nnz)
     rows = 40 * g.n_blocks
-    # two fp32 pooled tensors + the kept lists + scan partials, 256-byte aligned
-    assert ws >= rows * 128 * 4 * 2 + 40 * nnz * 4
-    assert ws < rows * 128 * 4 * 2 + 40 * nnz * 4 + 4096
+    nbp = (g.n_blocks + 31) // 32 * 32
+    # qbar [BH, Nb, D] + kbar transposed [BH, D, Nb padded to 32] (fp32) + the
+    # kept lists + scan partials, each 256-byte aligned
+    need = rows * 128 * 4 + 40 * 128 * nbp * 4 + 40 * nnz * 4
+    assert need <= ws < need + 4096

@@ -124,3 +124,23 @@ def test_monotone_in_rho_and_tau_on_gpu():
             if prev is not None:
                 assert all(a <= b for a, b in zip(prev, cur))
             prev = cur
+
+
+@pytest.mark.parametrize("name,gamma", [("tiny", None), ("wan13b_480p", None)])
+@pytest.mark.parametrize("mode,value", [("static", 0.2), ("dynamic", 0.8)])
+def test_selection_without_score_export_matches(name, gamma, mode, value):
+    # the bench path calls selection without exporting scores; static mode then
+    # skips scoring the forced blocks -- the kept CSR must not change
+    wl = WORKLOADS[name]
+    bits = make_qkv_bf16(wl, heads=range(min(wl.heads, 4)))
+    wl = Workload(wl.name, wl.batch, min(wl.heads, 4), wl.head_dim, wl.geom, wl.seed)
+    q, k, _ = gpu_inputs(bits)
+    cand = abi.dynrad_build_candidates(wl.geom)
+    rp1, col1, _ = abi.dynrad_select_blocks(q, k, wl.geom, cand, mode, value, scores=True)
+    rp1, col1 = rp1.clone(), col1.clone()
+    rp2, col2, _ = abi.dynrad_select_blocks(q, k, wl.geom, cand, mode, value, scores=False)
+    torch.cuda.synchronize()
+    check_device_status()
+    assert torch.equal(rp1, rp2)
+    n = int(rp1[-1])
+    assert torch.equal(col1[:n], col2[:n])
