@@ -36,6 +36,8 @@ EXPORTED = (
     "dynrad_sparse_attn",
     "dynrad_device_status",
     "dynrad_status_string",
+    "dynrad_static_scratch_bytes",
+    "dynrad_select_blocks_static_scratch",
 )
 
 
@@ -97,6 +99,12 @@ def lib() -> ctypes.CDLL:
         L.dynrad_device_status.argtypes = [_I32P, _I32, _VP]
         L.dynrad_status_string.restype = ctypes.c_char_p
         L.dynrad_status_string.argtypes = [_I32]
+        L.dynrad_static_scratch_bytes.restype = _SZ
+        L.dynrad_static_scratch_bytes.argtypes = []
+        L.dynrad_select_blocks_static_scratch.restype = ctypes.c_int
+        L.dynrad_select_blocks_static_scratch.argtypes = [_VP, _VP, _I32, _I32, _I32, _I32, _GP, _VP, _VP, _I64,
+                                                          _I64, _VP, _VP, _I32, ctypes.c_double, _VP, _VP, _I64,
+                                                          _VP, _VP]
         _lib = L
     return _lib
 
@@ -225,6 +233,21 @@ def dynrad_sparse_attn(q, k, v, block, row_ptr, col_idx, scale=0.0, out=None, ls
                                     _ptr(col_idx), float(scale), _ptr(o), _ptr(lse_t), _stream(stream)),
            "dynrad_sparse_attn")
     return o, lse_t
+
+
+def dynrad_select_blocks_static_scratch(q, k, geom, cand, mode, value, row_ptr, col_idx, scores=None,
+                                        stream=None) -> None:
+    """Stage 2 into caller-provided outputs, with the library's built-in device
+    scratch instead of a workspace: the call allocates nothing (for callers
+    that cannot allocate device memory).  Calls that overlap on the GPU race."""
+    _require_cuda(q, k, row_ptr, col_idx, scores)
+    B, H, N, D = q.shape
+    L = lib()
+    _check(L.dynrad_select_blocks_static_scratch(
+        _ptr(q), _ptr(k), B, H, N, D, ctypes.byref(make_geom(geom)), _ptr(cand["row_ptr"]), _ptr(cand["col"]),
+        cand["nnz"], cand["max_row"], _ptr(cand["forced_lo"]), _ptr(cand["forced_hi"]),
+        MODES[mode] if isinstance(mode, str) else mode, float(value), _ptr(row_ptr), _ptr(col_idx),
+        col_idx.numel(), _ptr(scores), _stream(stream)), "dynrad_select_blocks_static_scratch")
 
 
 def dynrad_device_status(clear: bool = True, stream=None) -> int:

@@ -361,3 +361,54 @@ int dynrad_sparse_attn(const void* q, const void* k, const void* v, int32_t B, i
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Stage 2 without a caller-provided workspace.
+//
+// Some callers cannot call cudaMalloc: a host library embedded in an
+// application whose caching allocator owns all device memory, or code that must
+// not risk the device-wide synchronisation a cudaMalloc / cudaFree may cause.
+// For them the selection scratch lives in this file-scope device array.  Every
+// GPU that loads the library holds it until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = static_cast<size_t>(32) << 20;  // 32 MiB
+
+static __device__ __align__(256) unsigned char g_select_scratch[kStaticScratchBytes];
+
+// Device address of g_select_scratch per device ordinal, resolved on the first
+// call on that device (the array's name in host code is only a stand-in).
+std::mutex g_scratch_mu;
+void* g_scratch_addr[256] = {};
+
+}  // namespace
+
+extern "C" size_t dynrad_static_scratch_bytes(void) { return kStaticScratchBytes; }
+
+extern "C" int dynrad_select_blocks_static_scratch(
+    const void* q, const void* k, int32_t B, int32_t H, int32_t N, int32_t D, const dynrad_geom* geom,
+    const int32_t* cand_row_ptr, const int32_t* cand_col, int64_t cand_nnz, int64_t cand_max_row,
+    const int32_t* forced_lo, const int32_t* forced_hi, int32_t mode, double rho_or_tau, int32_t* row_ptr,
+    int32_t* col_idx, int64_t col_cap, float* scores_out, dynrad_stream_t stream) {
+  const size_t need = dynrad_select_workspace_bytes(B, H, N, D, geom, cand_nnz);
+  if (need == 0) return DYNRAD_ERR_INVALID_ARG;
+  if (need > kStaticScratchBytes) return DYNRAD_ERR_CAPACITY;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return DYNRAD_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_addr[dev] == nullptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || p == nullptr) return DYNRAD_ERR_CUDA;
+      g_scratch_addr[dev] = p;
+    }
+    scratch = g_scratch_addr[dev];
+  }
+  // The scratch needs no clearing: every byte the selection reads in it is
+  // written earlier in the same call.
+  return dynrad_select_blocks(q, k, B, H, N, D, geom, cand_row_ptr, cand_col, cand_nnz, cand_max_row, forced_lo,
+                              forced_hi, mode, rho_or_tau, row_ptr, col_idx, col_cap, scores_out, scratch, need,
+                              stream);
+}

@@ -153,6 +153,38 @@ int dynrad_select_blocks(const void *q, const void *k, int32_t B, int32_t H,
                          size_t workspace_bytes, dynrad_stream_t stream);
 
 /*
+ * Stage 2 for callers that cannot allocate device memory (no counterpart in the
+ * paper).  A host library that runs inside an application whose own caching
+ * allocator owns the device's memory, or that must not risk the device-wide
+ * synchronisation cudaMalloc / cudaFree can cause, has no way to provide the
+ * workspace dynrad_select_blocks wants.  This call is dynrad_select_blocks with
+ * the workspace taken from a device array built into the library:
+ * dynrad_static_scratch_bytes() bytes (32 MiB) on every GPU that loads the
+ * library, held until the process exits.  The caller still provides every input
+ * and output buffer; the call allocates nothing and calls no allocating routine.
+ *
+ *   Arguments, layouts and results: as dynrad_select_blocks, without
+ *   workspace / workspace_bytes.
+ *   Errors: DYNRAD_ERR_CAPACITY when dynrad_select_workspace_bytes(...) exceeds
+ *   dynrad_static_scratch_bytes() (e.g. B=1, H=12, 32,760 tokens, block 64 fits;
+ *   H=40 at 75,600 tokens does not); DYNRAD_ERR_INVALID_ARG for arguments the
+ *   workspace size cannot be computed for; otherwise as dynrad_select_blocks.
+ *   The first call on a device looks up the array's device address (with that
+ *   device current); make that first call before any stream capture.
+ *   All calls on a device share the one array and it keeps the last call's
+ *   contents: calls that overlap on the GPU (other streams, other host threads)
+ *   race and corrupt each other's results.  Serialise them.
+ */
+size_t dynrad_static_scratch_bytes(void);
+int dynrad_select_blocks_static_scratch(
+    const void *q, const void *k, int32_t B, int32_t H, int32_t N, int32_t D,
+    const dynrad_geom *geom, const int32_t *cand_row_ptr,
+    const int32_t *cand_col, int64_t cand_nnz, int64_t cand_max_row,
+    const int32_t *forced_lo, const int32_t *forced_hi, int32_t mode,
+    double rho_or_tau, int32_t *row_ptr, int32_t *col_idx, int64_t col_cap,
+    float *scores_out, dynrad_stream_t stream);
+
+/*
  * Stage 3: block-sparse attention forward (Eq. 13 with epsilon -> 0).
  *
  * For every (b, h) and query token q of block I:
