@@ -36,6 +36,7 @@ EXPORTED = (
     "dynrad_sparse_attn",
     "dynrad_device_status",
     "dynrad_status_string",
+    "dynrad_debug_exp2",
     "dynrad_static_scratch_bytes",
     "dynrad_select_blocks_static_scratch",
 )
@@ -99,6 +100,8 @@ def lib() -> ctypes.CDLL:
         L.dynrad_device_status.argtypes = [_I32P, _I32, _VP]
         L.dynrad_status_string.restype = ctypes.c_char_p
         L.dynrad_status_string.argtypes = [_I32]
+        L.dynrad_debug_exp2.restype = ctypes.c_int
+        L.dynrad_debug_exp2.argtypes = [_VP, _VP, _VP, _I64, _VP]
         L.dynrad_static_scratch_bytes.restype = _SZ
         L.dynrad_static_scratch_bytes.argtypes = []
         L.dynrad_select_blocks_static_scratch.restype = ctypes.c_int
@@ -248,6 +251,15 @@ def dynrad_select_blocks_static_scratch(q, k, geom, cand, mode, value, row_ptr, 
         cand["nnz"], cand["max_row"], _ptr(cand["forced_lo"]), _ptr(cand["forced_hi"]),
         MODES[mode] if isinstance(mode, str) else mode, float(value), _ptr(row_ptr), _ptr(col_idx),
         col_idx.numel(), _ptr(scores), _stream(stream)), "dynrad_select_blocks_static_scratch")
+
+
+def dynrad_debug_exp2(x: torch.Tensor):
+    """(approximation, CUDA exp2f) of 2^x for a float32 CUDA tensor."""
+    _require_cuda(x)
+    poly = torch.empty_like(x)
+    ref = torch.empty_like(x)
+    _check(lib().dynrad_debug_exp2(_ptr(x), _ptr(poly), _ptr(ref), x.numel(), _stream()), "dynrad_debug_exp2")
+    return poly, ref
 
 
 def dynrad_device_status(clear: bool = True, stream=None) -> int:

@@ -1,32 +1,41 @@
 // Stage 3: block-sparse attention forward on the 5th-generation tensor cores
 // (DynamicRad, Sec. 3.3, Eqs. 12-13 with epsilon -> 0).
 //
-// One CTA computes one tile of 128 query rows (R = 128 / B_s query blocks) of
-// one (batch, head).  It walks the ascending union of the R rows' kept-block
-// lists in key steps of KW = min(B_s, 64) keys (a 128-key block is two steps);
-// the rows whose own list lacks the current block are masked to -inf.
+// One CTA (one per SM) computes 256 query rows of one (batch, head) as two
+// 128-row tiles that share one stream of K / V tiles: R = 256 / B_s query
+// blocks.  The producer walks the ascending union of the R rows' kept-block
+// lists and packs consecutive union blocks into 128-key steps (two 64-key
+// blocks, four 32-key blocks, or one 128-key block), so every Q K^T is a
+// 128 x 128 x D product -- the shape at which tcgen05 runs at its full rate
+// (N = 64 runs at two thirds of it).  A tile none of whose query blocks keeps
+// any block of the step skips its tensor-core work for that step; inside an
+// active tile the (row, block) pairs outside a row's own list are masked.
 //
-// Two CTAs share an SM (256 tensor-memory columns and < 113 KB of shared memory
-// each), so the softmax of one overlaps the tensor-core work of the other.
+// Warp roles (320 threads):
+//   warps 0-3, 4-7  softmax of tile 0 / tile 1: thread t of the warpgroup owns
+//              query row t of its tile = TMEM lane t.  Reads S = Q K^T (128
+//              columns) twice -- once for the row max, once for the exponentials,
+//              64 columns at a time to bound registers -- keeps the running
+//              max / sum in fp32 (lazy rescale: O is
+//              rescaled only when the row max grows by more than 2^8), writes
+//              P = 2^(...) as bf16 pairs over the first 64 columns of its S
+//              buffer, and finally normalises O and writes O and the
+//              log-sum-exp.  One exponential pair in four is computed on the FMA
+//              pipe (common.cuh exp2_poly2) to unload the MUFU unit.
+//   warp 8     producer: merges the R sorted CSR rows, publishes each step's
+//              block list, and issues TMA loads of the two Q tiles and of the
+//              K and V tiles of every step (128-byte swizzled, non-multicast)
+//              into a ring of single-tile slots.
+//   warp 9     MMA issuer (one thread), per tile t and step j:
+//              O_t += P_t(j) V(j) (A = P from tensor memory, B = V from shared
+//              memory, MN-major), then S_t = Q_t K(j+1)^T (A, B from shared
+//              memory).  Both go to the tensor core in this issue order, so the
+//              Q K^T that overwrites S_t runs after the P V product that reads
+//              P_t from the same columns; its completion also tells the softmax
+//              that O_t is up to date before a rescale.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax: thread t owns query row t of the tile = TMEM lane t.
-//              Loads S = Q K^T from tensor memory, releases it at once (the
-//              next Q K^T may overwrite it while the exponentials run), keeps
-//              the running max / sum in fp32 (lazy rescale: O is rescaled only
-//              when the row max grows by more than 2^8), writes P = 2^(...) as
-//              bf16 into tensor memory, and finally normalises O and writes O
-//              and the log-sum-exp.
-//   warp 4     producer: merges the R sorted CSR rows and issues TMA loads of the
-//              Q tile and of the K / V key steps (128-byte swizzled,
-//              non-multicast) into a STAGES-deep shared-memory ring.
-//   warp 5     MMA issuer (one thread): S = Q K^T (A and B from shared memory)
-//              and O += P V (A = P from tensor memory, B = V from shared memory,
-//              MN-major); fp32 accumulators in tensor memory.
-//
-// Tensor memory (256 columns): O [0, D), S [128, 128 + KW), P0 / P1 (KW / 2
-// columns each, bf16 pairs) at 192 / 224.  P is double-buffered so the
-// softmax of step j+1 need not wait for the P V product of step j.
+// Tensor memory (512 columns): O_t at 128 t (D columns), S_t at 256 + 128 t
+// (128 columns; P_t over its first 64).
 //
 // Every wait is bounded (common.cuh): a wait that runs out records
 // DYNRAD_ERR_DEVICE, raises a CTA-wide abort flag, and all roles unwind to the
@@ -39,23 +48,29 @@ namespace dynrad {
 
 template <int D, int BS>
 struct AttnCfg {
-  static constexpr int kM = 128;
-  static constexpr int kR = kM / BS;                 // query blocks per tile
-  static constexpr int kKW = BS < 64 ? BS : 64;      // keys per step
-  static constexpr int kSub = BS / kKW;              // steps per kept block
+  static constexpr int kTiles = 2;                   // 128-row query tiles per CTA
+  static constexpr int kM = 128;                     // rows per tile
+  static constexpr int kR = kTiles * kM / BS;        // query blocks per CTA
+  static constexpr int kRT = kM / BS;                // query blocks per tile
+  static constexpr int kKeys = 128;                  // keys per step
+  static constexpr int kBPS = kKeys / BS;            // kept blocks per step
   static constexpr int kChunks = D / 64;             // 128-byte column chunks
-  static constexpr int kQBytes = kM * D * 2;
-  static constexpr int kKVBytes = kKW * D * 2;       // one K (or V) step
-  static constexpr int kStagesRaw = (98304 - kQBytes) / (2 * kKVBytes);
-  static constexpr int kStages = kStagesRaw < 2 ? 2 : (kStagesRaw > 6 ? 6 : kStagesRaw);
-  static constexpr int kSmemData = kQBytes + kStages * 2 * kKVBytes;
-  static constexpr int kSmemCtrl = 512;
-  static constexpr int kSmemTotal = kSmemData + kSmemCtrl + 1024;  // +1024: manual alignment
-  static constexpr uint32_t kColO = 0, kColS = 128, kColP0 = 192, kColP1 = 224;
-  static constexpr uint32_t kTmemCols = 256;
+  static constexpr int kQTileBytes = kM * D * 2;
+  static constexpr int kTileBytes = kKeys * D * 2;   // one K or one V tile of a step
+  static constexpr int kMetaSlots = 8;
+  static constexpr int kSmemCtrl = 1024;
+  static constexpr int kSmemBudget = 227 * 1024 - kSmemCtrl - 1024;  // 1024: manual alignment
+  static constexpr int kSlotsRaw = (kSmemBudget - kTiles * kQTileBytes) / kTileBytes;
+  static constexpr int kSlots = kSlotsRaw < 3 ? 3 : (kSlotsRaw > 8 ? 8 : kSlotsRaw);
+  static constexpr int kSmemData = kTiles * kQTileBytes + kSlots * kTileBytes;
+  static constexpr int kSmemTotal = kSmemData + kSmemCtrl + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  __host__ __device__ static constexpr uint32_t col_o(int t) { return 128u * t; }
+  __host__ __device__ static constexpr uint32_t col_s(int t) { return 256u + 128u * t; }
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(BS == 32 || BS == 64 || BS == 128, "block size");
-  static_assert(2 * kSmemTotal <= 227 * 1024, "two CTAs per SM");
+  static_assert(kR <= 32, "one producer lane per query block");
+  static_assert(kSmemTotal <= 227 * 1024, "shared memory");
 };
 
 struct AttnParams {
@@ -68,9 +83,12 @@ struct AttnParams {
   float scale_log2;   // logit scale * log2(e)
 };
 
-struct RingEntry {
-  int32_t key0;       // first key token of the step, -1 = end of the walk
-  uint32_t mask;      // bit r: query block I0 + r keeps the step's block
+// One 128-key step: up to 4 kept blocks; nblk = 0 ends the walk.
+struct StepMeta {
+  int32_t key0[4];    // first key token of each block
+  uint32_t mask[4];   // bit r: query block I0 + r keeps that block
+  int32_t nblk;
+  int32_t pad;
 };
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -80,58 +98,55 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 }
 
 template <int D, int BS>
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(320, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = AttnCfg<D, BS>;
-  constexpr int S = C::kStages;
-  constexpr int KW = C::kKW;
+  constexpr int NS = C::kSlots;
+  constexpr int MS = C::kMetaSlots;
+  constexpr int BPS = C::kBPS;
+  constexpr uint32_t kTileMask = (1u << C::kRT) - 1u;
   extern __shared__ uint8_t attn_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(attn_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* q_smem = smem;
-  uint8_t* kv_smem = smem + C::kQBytes;  // stage s: K at 2s, V at 2s+1
+  uint8_t* q_smem = smem;                                 // tile t at t * kQTileBytes
+  uint8_t* slot_smem = smem + C::kTiles * C::kQTileBytes;  // load i (K_j: 2j, V_j: 2j+1) in slot i % NS
   uint8_t* ctrl = smem + C::kSmemData;
   uint64_t* bar = reinterpret_cast<uint64_t*>(ctrl);
   uint64_t* q_full = bar;
-  uint64_t* k_full = bar + 1;
-  uint64_t* v_full = k_full + S;
-  uint64_t* kv_empty = v_full + S;
-  uint64_t* s_full = kv_empty + S;
-  uint64_t* s_free = s_full + 1;
-  uint64_t* p_full = s_free + 1;     // [2]
-  uint64_t* pv_done = p_full + 2;    // [2]
-  uint64_t* drain = pv_done + 2;
-  RingEntry* ring = reinterpret_cast<RingEntry*>(drain + 1);
-  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(ring + S);
+  uint64_t* slot_full = bar + 1;
+  uint64_t* slot_empty = slot_full + NS;
+  uint64_t* meta_full = slot_empty + NS;   // [MS]
+  uint64_t* s_full = meta_full + MS;       // [tile]
+  uint64_t* p_full = s_full + 2;           // [tile]
+  uint64_t* drain = p_full + 2;
+  StepMeta* meta = reinterpret_cast<StepMeta*>(drain + 1);
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(meta + MS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_s + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x;
   const int bh = blockIdx.y;
-  const int I0 = tile * C::kR;
+  const int I0 = blockIdx.x * C::kR;
   const int q_row0 = I0 * BS;
   const int nb = p.nb;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&slot_full[s], 1);
+      mbar_init(&slot_empty[s], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 128);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&p_full[b], 128);
-      mbar_init(&pv_done[b], 1);
+    for (int m = 0; m < MS; ++m) mbar_init(&meta_full[m], 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_base_s, C::kTmemCols);
     tmem_relinquish();
   }
@@ -140,7 +155,7 @@ __global__ void __launch_bounds__(192, 2)
   tc_fence_after();
   const uint32_t taddr = *tmem_base_s;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------- producer
     int32_t ptr = 0, end = 0, cur = INT32_MAX;
     if (lane < C::kR && I0 + lane < nb) {
@@ -158,122 +173,172 @@ __global__ void __launch_bounds__(192, 2)
       prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
-      mbar_arrive_expect_tx(q_full, C::kQBytes);
+      mbar_arrive_expect_tx(q_full, C::kTiles * C::kQTileBytes);
 #pragma unroll
-      for (int c = 0; c < C::kChunks; ++c)
-        tma_load_3d(q_smem + c * (C::kM * 128), &tm_q, q_full, c * 64, q_row0, bh);
+      for (int t = 0; t < C::kTiles; ++t)
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_3d(q_smem + t * C::kQTileBytes + c * (C::kM * 128), &tm_q, q_full, c * 64,
+                      q_row0 + t * C::kM, bh);
     }
-    int j = 0;  // steps issued
-    bool ok = true, done = false;
-    while (!done) {
-      int32_t m = cur;
+    bool ok = true;
+    int li = 0;  // loads issued (K_j = 2j, V_j = 2j + 1, end marker = 2n)
+    // waits (bounded) until slot li % NS is free again
+    auto slot_ready = [&](int i) -> bool {
+      bool w = true;
+      if (i >= NS && lane == 0) w = mbar_wait(&slot_empty[i % NS], ((i / NS) - 1) & 1, abort_flag);
+      return __shfl_sync(0xffffffffu, w, 0);
+    };
+    for (int j = 0;; ++j) {
+      // gather the step's blocks: the next BPS union members
+      StepMeta st;
+      st.nblk = 0;
+      st.pad = 0;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) m = min(m, __shfl_xor_sync(0xffffffffu, m, off));
-      const bool mine = lane < C::kR && cur == m && m != INT32_MAX;
-      const uint32_t mask = __ballot_sync(0xffffffffu, mine);
-      if (mine) {
-        // advance past m, skipping malformed entries (out of range or not ascending)
-        ++ptr;
-        cur = INT32_MAX;
-        while (ptr < end) {
-          const int32_t c = p.col_idx[ptr];
-          if (c > m && c < nb) { cur = c; break; }
-          record_error(DYNRAD_ERR_DEVICE);
-          ++ptr;
-        }
+      for (int b = 0; b < 4; ++b) {
+        st.key0[b] = 0;
+        st.mask[b] = 0u;
       }
-      // the kept block's key steps (one, or two halves of a 128-key block);
-      // a step entirely past the sequence end is skipped
-      const int nsub = (m == INT32_MAX) ? 1 : C::kSub;
-      for (int sub = 0; sub < nsub; ++sub) {
-        const int key0 = (m == INT32_MAX) ? -1 : m * BS + sub * KW;
-        if (key0 >= p.N) continue;
-        const int s = j % S;
-        if (j >= S) {
-          bool w = true;
-          if (lane == 0) w = mbar_wait(&kv_empty[s], ((j / S) - 1) & 1, abort_flag);
-          w = __shfl_sync(0xffffffffu, w, 0);
-          if (!w) { ok = false; done = true; break; }
+#pragma unroll
+      for (int b = 0; b < BPS; ++b) {
+        int32_t m = cur;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = min(m, __shfl_xor_sync(0xffffffffu, m, off));
+        const bool mine = lane < C::kR && cur == m && m != INT32_MAX;
+        const uint32_t mask = __ballot_sync(0xffffffffu, mine);
+        if (mine) {
+          // advance past m, skipping malformed entries (out of range or not ascending)
+          ++ptr;
+          cur = INT32_MAX;
+          while (ptr < end) {
+            const int32_t c = p.col_idx[ptr];
+            if (c > m && c < nb) { cur = c; break; }
+            record_error(DYNRAD_ERR_DEVICE);
+            ++ptr;
+          }
         }
+        // once the union is exhausted every later slot is empty too, so slot b
+        // holds the b-th block of the step
+        st.key0[b] = m != INT32_MAX ? m * BS : 0;
+        st.mask[b] = m != INT32_MAX ? mask : 0u;
+        st.nblk += m != INT32_MAX ? 1 : 0;
+      }
+      // publish the step (the walk ends with nblk = 0)
+      if (!slot_ready(li)) { ok = false; break; }
+      if (lane == 0) {
+        meta[j % MS] = st;
+        mbar_arrive(&meta_full[j % MS]);
+      }
+      if (st.nblk == 0) {
+        if (lane == 0) mbar_arrive(&slot_full[li % NS]);  // end marker in the K position
+        __syncwarp();
+        break;
+      }
+      // K tile then V tile; blocks missing at the end of the walk repeat the
+      // first block so the tile holds finite data (its columns are masked)
+#pragma unroll
+      for (int kv = 0; kv < 2; ++kv) {
+        if (kv == 1 && !slot_ready(li)) { ok = false; break; }
         if (lane == 0) {
-          ring[s].key0 = key0;
-          ring[s].mask = mask;
-          if (key0 < 0) {
-            mbar_arrive(&k_full[s]);
-          } else {
-            uint8_t* ks = kv_smem + (2 * s) * C::kKVBytes;
-            uint8_t* vs = kv_smem + (2 * s + 1) * C::kKVBytes;
-            mbar_arrive_expect_tx(&k_full[s], C::kKVBytes);
+          uint8_t* dst = slot_smem + (li % NS) * C::kTileBytes;
+          const CUtensorMap* map = kv == 0 ? &tm_k : &tm_v;
+          mbar_arrive_expect_tx(&slot_full[li % NS], C::kTileBytes);
+#pragma unroll
+          for (int b = 0; b < BPS; ++b) {
+            const int key0 = b < st.nblk ? st.key0[b] : st.key0[0];
 #pragma unroll
             for (int c = 0; c < C::kChunks; ++c)
-              tma_load_3d(ks + c * (KW * 128), &tm_k, &k_full[s], c * 64, key0, bh);
-            mbar_arrive_expect_tx(&v_full[s], C::kKVBytes);
-#pragma unroll
-            for (int c = 0; c < C::kChunks; ++c)
-              tma_load_3d(vs + c * (KW * 128), &tm_v, &v_full[s], c * 64, key0, bh);
+              tma_load_3d(dst + c * (C::kKeys * 128) + b * (BS * 128), map, &slot_full[li % NS], c * 64,
+                          key0, bh);
           }
         }
         __syncwarp();
-        ++j;
-        if (key0 < 0) { done = true; break; }
+        ++li;
       }
+      if (!ok) break;
     }
     if (!ok && lane == 0) {
       // unwinding: let the copies already issued land before shared memory is
       // given back (bounded; ignores the abort flag)
-      for (int i = (j > S ? j - S : 0); i < j; ++i) {
-        mbar_wait(&k_full[i % S], (i / S) & 1, nullptr);
-        mbar_wait(&v_full[i % S], (i / S) & 1, nullptr);
-      }
+      for (int i = (li > NS ? li - NS : 0); i < li; ++i) mbar_wait(&slot_full[i % NS], (i / NS) & 1, nullptr);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, KW, false, false);
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, C::kKeys, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
       const uint32_t q_base = smem_u32(q_smem);
-      const uint32_t kv_base = smem_u32(kv_smem);
+      const uint32_t slot_base = smem_u32(slot_smem);
       bool ok = mbar_wait(q_full, 0, abort_flag);
-      int j = 0;
-      auto issue_pv = [&](int i) -> bool {
-        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(&v_full[i % S], (i / S) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t v_addr = kv_base + (2 * (i % S) + 1) * C::kKVBytes;
-        const uint32_t p_col = (i & 1) ? C::kColP1 : C::kColP0;
+      bool started[2] = {false, false};   // O_t holds a P V product
+      auto tile_act = [&](const StepMeta& m, int t) -> bool {
+        uint32_t any = 0;
 #pragma unroll
-        for (int kk = 0; kk < KW / 16; ++kk) {
-          // V step [KW keys][D] as the MN-major B operand: 64-column chunks
-          // KW*128 bytes apart (leading offset), 8-key groups 1024 bytes apart
-          const uint64_t bdesc = smem_desc_sw128(v_addr + kk * 2048, KW * 128, 1024);
-          mma_ts(taddr + C::kColO, taddr + p_col + kk * 8, bdesc, idesc_pv,
-                 (i > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&kv_empty[i % S]);
-        mma_commit(&pv_done[i & 1]);
-        return true;
+        for (int b = 0; b < BPS; ++b) any |= (b < m.nblk) ? m.mask[b] : 0u;
+        return ((any >> (t * C::kRT)) & kTileMask) != 0u;
       };
-      while (ok) {
-        const int s = j % S;
-        if (!mbar_wait(&k_full[s], (j / S) & 1, abort_flag)) { ok = false; break; }
-        const RingEntry e = ring[s];
-        if (e.key0 < 0) break;
-        // S is single-buffered: the softmax must have read S_{j-1}
-        if (j >= 1 && !mbar_wait(s_free, (j - 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t k_addr = kv_base + (2 * s) * C::kKVBytes;
+      auto issue_qk = [&](int t, int i) {   // S_t = Q_t K^T, K in load slot i
+        const uint32_t qt = q_base + t * C::kQTileBytes;
+        const uint32_t kb = slot_base + (i % NS) * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int c = kk >> 2, off = (kk & 3) * 32;
-          const uint64_t adesc = smem_desc_sw128(q_base + c * (C::kM * 128) + off, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(k_addr + c * (KW * 128) + off, 16, 1024);
-          mma_ss(taddr + C::kColS, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+          const uint64_t adesc = smem_desc_sw128(qt + c * (C::kM * 128) + off, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(kb + c * (C::kKeys * 128) + off, 16, 1024);
+          mma_ss(taddr + C::col_s(t), adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        mma_commit(s_full);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+      };
+      auto issue_pv = [&](int t, int i) {   // O_t += P_t V, V in load slot i
+        const uint32_t vb = slot_base + (i % NS) * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < C::kKeys / 16; ++kk) {
+          // V tile [128 keys][D] as the MN-major B operand: 64-column chunks
+          // 128*128 bytes apart (leading offset), 8-key groups 1024 bytes apart
+          const uint64_t bdesc = smem_desc_sw128(vb + kk * 2048, C::kKeys * 128, 1024);
+          mma_ts(taddr + C::col_o(t), taddr + C::col_s(t) + kk * 8, bdesc, idesc_pv,
+                 (started[t] || kk > 0) ? 1u : 0u);
+        }
+        started[t] = true;
+      };
+      // step 0: S_t = Q_t K(0)^T
+      int j = 0;
+      StepMeta cur_m;
+      if (ok && !mbar_wait(&slot_full[0], 0, abort_flag)) ok = false;
+      if (ok) {
+        cur_m = meta[0];
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t) {
+          if (cur_m.nblk > 0 && tile_act(cur_m, t)) issue_qk(t, 0);
+          mma_commit(&s_full[t]);
+        }
+        if (cur_m.nblk > 0) mma_commit(&slot_empty[0]);
+      }
+      while (ok && cur_m.nblk > 0) {
+        const int iv = 2 * j + 1, ik = 2 * j + 2;   // V(j) and K(j+1) load indices
+        if (!mbar_wait(&slot_full[iv % NS], (iv / NS) & 1, abort_flag)) { ok = false; break; }
+        StepMeta next_m;
+        bool have_next = false;
+        for (int t = 0; t < 2; ++t) {
+          // O_t += P_t(j) V(j) once the softmax has written P_t(j)
+          if (!mbar_wait(&p_full[t], j & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          if (tile_act(cur_m, t)) issue_pv(t, iv);
+          if (t == 1) mma_commit(&slot_empty[iv % NS]);
+          // S_t = Q_t K(j+1)^T (after the P V above in issue order)
+          if (!have_next) {
+            if (!mbar_wait(&slot_full[ik % NS], (ik / NS) & 1, abort_flag)) { ok = false; break; }
+            next_m = meta[(j + 1) % MS];
+            have_next = true;
+            tc_fence_after();
+          }
+          if (next_m.nblk > 0 && tile_act(next_m, t)) issue_qk(t, ik);
+          if (t == 1 && next_m.nblk > 0) mma_commit(&slot_empty[ik % NS]);
+          mma_commit(&s_full[t]);
+        }
+        if (!ok) break;
+        cur_m = next_m;
         ++j;
       }
-      if (ok && j >= 1) issue_pv(j - 1);
       // all issued tensor-core work finished before tensor memory is released
       mma_commit(drain);
       mbar_wait(drain, 0, nullptr);
@@ -281,140 +346,173 @@ __global__ void __launch_bounds__(192, 2)
     __syncwarp();
   } else {
     // -------------------------------------------------------------- softmax
-    const int t = threadIdx.x;             // tile row = TMEM lane
-    const int sub = t / BS;                // query block within the tile
-    const int row = q_row0 + t;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int tile = warp >> 2;                    // warpgroup = query tile
+    const int t = threadIdx.x - tile * 128;        // row within the tile = TMEM lane
+    const int mbit = tile * C::kRT + t / BS;       // this row's bit in the block masks
+    const int row = q_row0 + tile * C::kM + t;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t col_s = C::col_s(tile), col_o = C::col_o(tile);
     const float c2 = p.scale_log2;
     float m_used = -INFINITY;              // running max in log2 units
     float l = 0.f;
+    bool any_pv = false;                   // a P V product reached O of this tile
     int j = 0;
     bool ok = true;
     for (;; ++j) {
-      const int s = j % S;
-      if (!__all_sync(0xffffffffu, mbar_wait(&k_full[s], (j / S) & 1, abort_flag))) { ok = false; break; }
-      const RingEntry e = ring[s];
-      if (e.key0 < 0) break;
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full, j & 1, abort_flag))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&meta_full[j % MS], (j / MS) & 1, abort_flag))) { ok = false; break; }
+      const StepMeta st = meta[j % MS];
+      // S_t(j) -- or, at the end marker, completion of the last P V product
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[tile], j & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
-      float sv[KW];
+      if (st.nblk == 0) break;
+      uint32_t tile_any = 0, row_bits = 0;
 #pragma unroll
-      for (int c = 0; c < KW / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(taddr + lane_base + C::kColS + c * 32, r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(r[i]);
+      for (int b = 0; b < BPS; ++b) {
+        const uint32_t mk = b < st.nblk ? st.mask[b] : 0u;
+        tile_any |= mk;
+        row_bits |= ((mk >> mbit) & 1u) << b;
       }
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(s_free);                 // S may be overwritten now
-      const bool active = (e.mask >> sub) & 1u;
-      const int nvalid = min(KW, p.N - e.key0);
-      const bool full = nvalid == KW;
-      float mx = -INFINITY;
-      if (active) {
-        if (full) {
-          // four independent max chains, then combined
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      const bool tile_active = ((tile_any >> (tile * C::kRT)) & kTileMask) != 0u;
+      if (tile_active) {
+        any_pv = true;
+        // State of each 64-key half for this row: every key valid (kept block,
+        // inside the sequence), none valid (block not kept / no block), or
+        // mixed (a sequence tail, or 32-key blocks with different states).
+        // Rows of one warp share their query block, so these are warp-uniform.
+        uint32_t half_full = 0, half_none = 0;
 #pragma unroll
-          for (int i = 0; i < KW; i += 8) {
+        for (int h = 0; h < C::kKeys / 64; ++h) {
+          bool all = true, none = true;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) m4[u] = fmax3(m4[u], sv[i + 2 * u], sv[i + 2 * u + 1]);
+          for (int b = 0; b < BPS; ++b) {
+            if (b * BS >= (h + 1) * 64 || (b + 1) * BS <= h * 64) continue;  // slot outside the half
+            const bool kept = (row_bits >> b) & 1u;
+            const int lo = max(h * 64, b * BS) - b * BS, hi = min((h + 1) * 64, (b + 1) * BS) - b * BS;
+            const bool inside = st.key0[b] + hi <= p.N;
+            const bool any_in = st.key0[b] + lo < p.N;
+            all = all && kept && inside;
+            none = none && !(kept && any_in);
           }
-          mx = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < KW; ++i)
-            if (i < nvalid) mx = fmaxf(mx, sv[i]);
+          half_full |= (all ? 1u : 0u) << h;
+          half_none |= (none ? 1u : 0u) << h;
         }
-      }
-      const float m_new = active ? fmaxf(m_used, mx * c2) : m_used;
-      const bool need = active && m_used != -INFINITY && m_new > m_used + 8.0f;
-      if (__any_sync(0xffffffffu, need)) {
-        // rescale O: the previous P V product must have landed first
-        if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const float alpha = need ? ex2_approx(m_used - m_new) : 1.0f;
+        // pass 1: row max over the valid keys, 64 columns at a time
+        float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(taddr + lane_base + C::kColO + c * 32, r);
+        for (int h = 0; h < C::kKeys / 64; ++h) {
+          if ((half_none >> h) & 1u) continue;
+          float sv[64];
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t r[32];
+            tmem_ld32(taddr + lane_base + col_s + h * 64 + c * 32, r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(r[i]);
+          }
           tmem_wait_ld();
+          if ((half_full >> h) & 1u) {
+            float m4[4] = {mx, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(taddr + lane_base + C::kColO + c * 32, r);
+            for (int i = 0; i < 64; i += 8) {
+#pragma unroll
+              for (int u = 0; u < 4; ++u) m4[u] = fmax3(m4[u], sv[i + 2 * u], sv[i + 2 * u + 1]);
+            }
+            mx = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+              const int k = h * 64 + i, b = k / BS;
+              const bool v = ((row_bits >> b) & 1u) && (st.key0[b] + (k % BS) < p.N);
+              if (v) mx = fmaxf(mx, sv[i]);
+            }
+          }
         }
-        tmem_wait_st();
-        if (need) {
-          l *= alpha;
-          m_used = m_new;
+        const bool active = (half_none != (1u << (C::kKeys / 64)) - 1u);
+        const float m_new = active ? fmaxf(m_used, mx * c2) : m_used;
+        const bool need = active && m_used != -INFINITY && m_new > m_used + 8.0f;
+        if (__any_sync(0xffffffffu, need)) {
+          // rescale O: S_t(j) completing means every earlier P V product has too
+          const float alpha = need ? ex2_approx(m_used - m_new) : 1.0f;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(taddr + lane_base + col_o + c * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(taddr + lane_base + col_o + c * 32, r);
+          }
+          if (need) {
+            l *= alpha;
+            m_used = m_new;
+          }
         }
-      }
-      if (active && m_used == -INFINITY) m_used = m_new;
-      uint32_t pk[KW / 2];
-      if (active && full) {
-        const float2 cc = make_float2(c2, c2);
-        const float2 mm = make_float2(-m_used, -m_used);
+        if (active && m_used == -INFINITY) m_used = m_new;
+        // pass 2: P over the first 64 columns of S_t; keys 64h .. 64h+63 are
+        // re-read from columns 64h .. and written as bf16 pairs to columns
+        // 32h .., which hold keys already consumed
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                          make_float2(0.f, 0.f)};
+        const float2 cc = make_float2(c2, c2);
+        const float2 mm = make_float2(-m_used, -m_used);
 #pragma unroll
-        for (int i = 0; i < KW; i += 2) {
-          const float2 x = __ffma2_rn(make_float2(sv[i], sv[i + 1]), cc, mm);
-          const float2 pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          acc[(i >> 1) & 3] = __fadd2_rn(acc[(i >> 1) & 3], pe);
-          pk[i / 2] = pack_bf16x2(pe.x, pe.y);
+        for (int h = 0; h < C::kKeys / 64; ++h) {
+          uint32_t pk[32];
+          if ((half_none >> h) & 1u) {
+#pragma unroll
+            for (int q2 = 0; q2 < 32; ++q2) pk[q2] = 0u;
+          } else {
+            float sv[64];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              uint32_t r[32];
+              tmem_ld32(taddr + lane_base + col_s + h * 64 + c * 32, r);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(r[i]);
+            }
+            tmem_wait_ld();
+            if ((half_full >> h) & 1u) {
+#pragma unroll
+              for (int q2 = 0; q2 < 32; ++q2) {
+                const float2 x = __ffma2_rn(make_float2(sv[2 * q2], sv[2 * q2 + 1]), cc, mm);
+                // one pair in four on the FMA pipe, the rest on MUFU
+                const float2 pe = (q2 & 3) == 3 ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                acc[q2 & 3] = __fadd2_rn(acc[q2 & 3], pe);
+                pk[q2] = pack_bf16x2(pe.x, pe.y);
+              }
+            } else {
+#pragma unroll
+              for (int q2 = 0; q2 < 32; ++q2) {
+                const int k = h * 64 + 2 * q2;
+                const int b0 = k / BS, b1 = (k + 1) / BS;
+                const bool v0 = ((row_bits >> b0) & 1u) && (st.key0[b0] + (k % BS) < p.N);
+                const bool v1 = ((row_bits >> b1) & 1u) && (st.key0[b1] + ((k + 1) % BS) < p.N);
+                const float p0 = v0 ? ex2_approx(fmaf(sv[2 * q2], c2, -m_used)) : 0.f;
+                const float p1 = v1 ? ex2_approx(fmaf(sv[2 * q2 + 1], c2, -m_used)) : 0.f;
+                acc[q2 & 3] = __fadd2_rn(acc[q2 & 3], make_float2(p0, p1));
+                pk[q2] = pack_bf16x2(p0, p1);
+              }
+            }
+          }
+          tmem_st32(taddr + lane_base + col_s + h * 32, pk);
         }
         const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
         const float2 a = __fadd2_rn(a01, a23);
         l += a.x + a.y;
-      } else {
-        float rs = 0.f;
-#pragma unroll
-        for (int i = 0; i < KW; i += 2) {
-          const float p0 = (active && i < nvalid) ? ex2_approx(fmaf(sv[i], c2, -m_used)) : 0.f;
-          const float p1 = (active && i + 1 < nvalid) ? ex2_approx(fmaf(sv[i + 1], c2, -m_used)) : 0.f;
-          rs += p0 + p1;
-          pk[i / 2] = pack_bf16x2(p0, p1);
-        }
-        l += rs;
+        tmem_wait_st();
       }
-      // P buffer j&1 was last read by the P V product of step j-2
-      if (j >= 2) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-      }
-      const uint32_t p_col = (j & 1) ? C::kColP1 : C::kColP0;
-      if constexpr (KW == 32) {
-        tmem_st16(taddr + lane_base + p_col, pk);
-      } else {
-        tmem_st32(taddr + lane_base + p_col, *reinterpret_cast<const uint32_t(*)[32]>(pk));
-      }
-      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[j & 1]);
+      mbar_arrive(&p_full[tile]);
     }
-    const int n_steps = j;
     if (ok) {
-      bool have_o = n_steps > 0;
-      if (have_o) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[(n_steps - 1) & 1], ((n_steps - 1) >> 1) & 1,
-                                               abort_flag)))
-          have_o = false;
-        tc_fence_after();
-      }
+      const bool have_o = any_pv;     // the final s_full wait covered the last P V
       const float inv_l = l > 0.f ? 1.0f / l : 0.f;
       __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + row) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
         if (have_o) {
-          tmem_ld32(taddr + lane_base + C::kColO + c * 32, r);
+          tmem_ld32(taddr + lane_base + col_o + c * 32, r);
           tmem_wait_ld();
         } else {
 #pragma unroll
@@ -440,7 +538,7 @@ __global__ void __launch_bounds__(192, 2)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(taddr, C::kTmemCols);
+  if (warp == 9) tmem_dealloc(taddr, C::kTmemCols);
 }
 
 }  // namespace dynrad

@@ -119,10 +119,11 @@ int launch_attn(const void* q, const void* k, const void* v, int BH, int N, cons
                 const int32_t* col_idx, float scale, void* o, float* lse, cudaStream_t st) {
   using C = AttnCfg<D, BS>;
   CUtensorMap mq, mk, mv;
-  // K / V boxes are one key step (C::kKW rows), the unit the kernel's ring
-  // slots and transaction counts are sized for
-  if (!encode_map(&mq, q, D, N, BH, C::kM) || !encode_map(&mk, k, D, N, BH, C::kKW) ||
-      !encode_map(&mv, v, D, N, BH, C::kKW))
+  // K / V boxes are one kept block (BS rows); a slot stacks C::kBPS of them,
+  // the unit the kernel's slots and transaction counts are sized for
+  static_assert(C::kBPS * BS == C::kKeys, "a step is kBPS blocks");
+  if (!encode_map(&mq, q, D, N, BH, C::kM) || !encode_map(&mk, k, D, N, BH, BS) ||
+      !encode_map(&mv, v, D, N, BH, BS))
     return DYNRAD_ERR_CUDA;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
@@ -141,7 +142,7 @@ int launch_attn(const void* q, const void* k, const void* v, int BH, int N, cons
   p.scale_log2 = scale * 1.4426950408889634f;
   const int tiles = (p.nb + C::kR - 1) / C::kR;
   dim3 grid(tiles, BH);
-  sparse_attn_kernel<D, BS><<<grid, 192, C::kSmemTotal, st>>>(mq, mk, mv, p);
+  sparse_attn_kernel<D, BS><<<grid, 320, C::kSmemTotal, st>>>(mq, mk, mv, p);
   return launch_status();
 }
 
@@ -167,6 +168,35 @@ const char* dynrad_status_string(int32_t status) {
     case DYNRAD_ERR_DEVICE: return "device-side check or bounded wait failed";
     default: return "unknown status";
   }
+}
+
+}  // extern "C"
+
+namespace {
+__global__ void exp2_diag_kernel(const float* x, float* poly, float* ref, int64_t n) {
+  const int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 2;
+  if (i + 1 < n) {
+    const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
+    poly[i] = r.x;
+    poly[i + 1] = r.y;
+    ref[i] = exp2f(x[i]);
+    ref[i + 1] = exp2f(x[i + 1]);
+  } else if (i < n) {
+    poly[i] = exp2_poly2(make_float2(x[i], x[i])).x;
+    ref[i] = exp2f(x[i]);
+  }
+}
+}  // namespace
+
+extern "C" {
+
+int dynrad_debug_exp2(const float* x, float* poly_out, float* ref_out, int64_t n, dynrad_stream_t stream) {
+  if (x == nullptr || poly_out == nullptr || ref_out == nullptr || n < 0) return DYNRAD_ERR_INVALID_ARG;
+  if (n == 0) return DYNRAD_OK;
+  const int64_t threads = 256, pairs = (n + 1) / 2;
+  exp2_diag_kernel<<<static_cast<unsigned>((pairs + threads - 1) / threads), threads, 0, as_stream(stream)>>>(
+      x, poly_out, ref_out, n);
+  return launch_status();
 }
 
 int dynrad_device_status(int32_t* status_out, int32_t clear, dynrad_stream_t stream) {

@@ -216,6 +216,16 @@ int dynrad_sparse_attn(const void *q, const void *k, const void *v, int32_t B,
 int dynrad_device_status(int32_t *status_out, int32_t clear,
                          dynrad_stream_t stream);
 
+/*
+ * Diagnostic: evaluates, for n device floats x, the FMA-pipe approximation of
+ * 2^x that the attention kernel's softmax uses for part of its exponentials
+ * (poly_out) and CUDA's exp2f (ref_out), so the approximation can be checked
+ * against CUDA's own results.  Valid range of the approximation: x <= 64
+ * (inputs below -125 give 2^-125).  Device pointers; asynchronous.
+ */
+int dynrad_debug_exp2(const float *x, float *poly_out, float *ref_out,
+                      int64_t n, dynrad_stream_t stream);
+
 /* Static string for a status code ("ok", "invalid argument", ...). */
 const char *dynrad_status_string(int32_t status);
 

@@ -136,3 +136,19 @@ def test_tiny_end_to_end(mode, value):
     col_np = col.cpu().numpy().astype(np.int64)[: rp_np[-1]]
     o_ref, lse_ref = _oracle_all(bits, wl.geom.block, rp_np, col_np, 1, wl.heads)
     compare_attention(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, f"tiny {mode}")
+
+
+def test_fma_pipe_exp2_against_cuda_exp2f():
+    # the softmax computes one exponential in four with the FMA-pipe
+    # approximation; check it against CUDA's exp2f over the range the kernel
+    # feeds it (running-max-shifted logits: x <= 8 with lazy rescale)
+    x = torch.cat([torch.linspace(-124.0, 8.0, 2_000_001), torch.tensor([0.0, -0.5, 0.5, 7.999, -1e-7])])
+    x = x.float().cuda()
+    poly, ref = abi.dynrad_debug_exp2(x)
+    torch.cuda.synchronize()
+    rel = ((poly.double() - ref.double()) / ref.double()).abs()
+    assert float(rel.max()) < 8e-5
+    # far below the range the result is tiny and positive (no inf / nan)
+    low = torch.tensor([-1000.0, -200.0, -126.0], device="cuda")
+    pl, _ = abi.dynrad_debug_exp2(low)
+    assert bool(torch.isfinite(pl).all()) and float(pl.max()) < 1e-37
