@@ -22,7 +22,8 @@ using namespace dynrad;
 namespace {
 
 constexpr int kMaxFrames = 16384;
-constexpr int kMaxBlocks = 16384;    // Nb bound of the selection kernel's shared memory
+constexpr int kMaxBlocks = 16384;        // Nb bound of the scoring kernel's shared memory
+constexpr int kMaxRowCandidates = 1024;  // candidates per row held in a warp's registers
 
 inline cudaStream_t as_stream(dynrad_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -307,12 +308,18 @@ int dynrad_select_blocks(const void* q, const void* k, int32_t B, int32_t H, int
     sp.counts = row_ptr;
     sp.kept_tmp = kept;
     sp.scores_out = scores_out;
+    // without an export the workspace's per-candidate array holds the scores
+    // and then, row by row, the kept lists (a row's warp reads all its scores
+    // before it writes)
+    sp.scores = scores_out != nullptr ? scores_out : reinterpret_cast<float*>(kept);
+    sp.rows_bh = static_cast<int>(bh);
     sp.cand_nnz = cand_nnz;
     sp.N = N;
     sp.block = g.block;
     sp.nb = g.nb;
     sp.nbp = padded_blocks(g.nb);
     sp.max_row = (cand_max_row > 0 && cand_max_row < g.nb) ? static_cast<int>(cand_max_row) : g.nb;
+    if (sp.max_row > kMaxRowCandidates) return DYNRAD_ERR_UNSUPPORTED;
     sp.mode = mode;
     sp.value = rho_or_tau;
     sp.scale = 1.0f / std::sqrt(static_cast<float>(D));
@@ -323,18 +330,34 @@ int dynrad_select_blocks(const void* q, const void* k, int32_t B, int32_t H, int
     else
       pool_kernel<64><<<pgrid, kS2Threads, 0, st>>>(sp);
     if ((rc = launch_status()) != DYNRAD_OK) return rc;
-    const size_t smem = s2_smem_bytes(D, g.nb, sp.max_row);
-    if (smem > 227 * 1024) return DYNRAD_ERR_UNSUPPORTED;
-    const void* kern = D == 128 ? reinterpret_cast<const void*>(select_kernel<128>)
-                                : reinterpret_cast<const void*>(select_kernel<64>);
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+    // scoring: union of 8 rows per CTA, scores to their candidate positions
+    const size_t ssmem = score_smem_bytes(D, g.nb);
+    if (ssmem > 227 * 1024) return DYNRAD_ERR_UNSUPPORTED;
+    const void* skern = D == 128 ? reinterpret_cast<const void*>(score_kernel<128>)
+                                 : reinterpret_cast<const void*>(score_kernel<64>);
+    if (cudaFuncSetAttribute(skern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ssmem)) !=
         cudaSuccess)
       return DYNRAD_ERR_CUDA;
     const dim3 sgrid(nq, static_cast<unsigned>(bh));
     if (D == 128)
-      select_kernel<128><<<sgrid, kS2Threads, smem, st>>>(sp);
+      score_kernel<128><<<sgrid, kS2Threads, ssmem, st>>>(sp);
     else
-      select_kernel<64><<<sgrid, kS2Threads, smem, st>>>(sp);
+      score_kernel<64><<<sgrid, kS2Threads, ssmem, st>>>(sp);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+    // selection: one warp per row, candidates in registers
+    const unsigned rblocks = static_cast<unsigned>((rows + kSelWarps - 1) / kSelWarps);
+    const bool dyn = mode == DYNRAD_DYNAMIC_THRESHOLD;
+    const int e = sp.max_row <= 128 ? 4 : (sp.max_row <= 256 ? 8 : (sp.max_row <= 512 ? 16 : 32));
+#define DYNRAD_LAUNCH_SELECT(E_)                                               \
+  if (e == E_) {                                                               \
+    if (dyn) select_kernel<E_, true><<<rblocks, kSelWarps * 32, 0, st>>>(sp);  \
+    else select_kernel<E_, false><<<rblocks, kSelWarps * 32, 0, st>>>(sp);     \
+  }
+    DYNRAD_LAUNCH_SELECT(4)
+    DYNRAD_LAUNCH_SELECT(8)
+    DYNRAD_LAUNCH_SELECT(16)
+    DYNRAD_LAUNCH_SELECT(32)
+#undef DYNRAD_LAUNCH_SELECT
     if ((rc = launch_status()) != DYNRAD_OK) return rc;
   }
   // counts -> offsets, compaction

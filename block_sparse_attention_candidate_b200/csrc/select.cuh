@@ -65,7 +65,9 @@ struct Stage2Params {
   const int32_t* forced_hi;
   int32_t* counts;          // kept count per row (row_ptr before the scan)
   int32_t* kept_tmp;        // [BH, cand_nnz] kept lists at the candidate offsets
-  float* scores_out;        // nullable
+  float* scores_out;        // nullable (caller's export of the scores)
+  float* scores;            // [BH, cand_nnz] scores used by the selection
+  int rows_bh;              // B * H
   int64_t cand_nnz;
   int N;
   int block;
@@ -110,24 +112,6 @@ struct Reach {
     return dynamic ? static_cast<double>(base + w) >= tau_z : w >= k;
   }
 };
-
-// Per-warp selection scratch in shared memory: bins 2 x 256 u32, weights[cap]
-// u64, keys[cap] u32, flags[cap] u8, rounded to 16 bytes.
-__host__ __device__ constexpr size_t sel_warp_bytes(int cap) {
-  return (2048 + static_cast<size_t>(cap) * 13 + 15) & ~static_cast<size_t>(15);
-}
-
-// Shared memory of stage2_kernel: [qsT 8*D f32][bitmap][wprefix][ulist nb]
-// [S 8*nb f32 | pool transpose tile 8*D f32][per-warp selection scratch].
-__host__ __device__ constexpr size_t s2_head_bytes(int D, int nb) {
-  return static_cast<size_t>(kSelRows) * D * 4 + static_cast<size_t>((nb + 31) / 32) * 4 +
-         static_cast<size_t>((nb + 31) / 32 + 1) * 4 + static_cast<size_t>(nb) * 4;
-}
-__host__ __device__ constexpr size_t s2_smem_bytes(int D, int nb, int cap) {
-  return ((s2_head_bytes(D, nb) + static_cast<size_t>(kSelRows) * (nb > D ? nb : D) * 4 + 15) &
-          ~static_cast<size_t>(15)) +
-         kSelRows * sel_warp_bytes(cap);
-}
 
 // Pool item: warp w pools block 8*grp + w of one (tensor, head).
 template <int D>
@@ -184,92 +168,125 @@ __device__ __forceinline__ void pool_item(const Stage2Params& p, bool is_k, int 
   }
 }
 
-// Score + select item: rows I0 .. I0+7 of head bh.
+// Pool: one CTA per (tensor, head, 8 consecutive blocks); many CTAs per SM keep
+// enough loads in flight to run at HBM bandwidth.
 template <int D>
-__device__ __forceinline__ void score_item(const Stage2Params& p, int bh, int I0, uint8_t* sm) {
+__global__ void __launch_bounds__(kS2Threads, 4) pool_kernel(Stage2Params p) {
+  __shared__ __align__(16) float tile[kSelRows * D];
+  const int nq = (p.nb + kSelRows - 1) / kSelRows;
+  const int grp = blockIdx.x % nq;
+  const bool is_k = (blockIdx.x / nq) != 0;
+  pool_item<D>(p, is_k, blockIdx.y, grp, tile);
+}
+
+// ---------------------------------------------------------------------------
+// Scoring: one CTA per (head, 8 consecutive query blocks).  The union of the 8
+// candidate lists is scored once per key block (each kbar value read feeds 8
+// dot products); every row's scores go to its candidate positions in a global
+// array [BH, cand_nnz] (a row's position of block J = rank of J in the row's
+// sorted list, from per-row bitmaps and prefix popcounts).
+// ---------------------------------------------------------------------------
+__host__ __device__ constexpr size_t score_smem_bytes(int D, int nb) {
+  // qsT [D][8] f32, union bitmap + prefix, 8 row bitmaps + prefixes, 8 "needs a
+  // score" bitmaps, union list
+  return static_cast<size_t>(kSelRows) * D * 4 +
+         static_cast<size_t>((nb + 31) / 32) * 4 * (2 + 3 * kSelRows) + static_cast<size_t>(nb) * 4 + 64;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kS2Threads, 3) score_kernel(Stage2Params p) {
+  extern __shared__ __align__(16) uint8_t sc_smem[];
   const int nb = p.nb;
   const int nwords = (nb + 31) >> 5;
-  const int cap = p.max_row;
-  float* qsT = reinterpret_cast<float*>(sm);                              // [D][8]
-  uint32_t* bitmap = reinterpret_cast<uint32_t*>(qsT + kSelRows * D);     // [nwords]
-  int32_t* wprefix = reinterpret_cast<int32_t*>(bitmap + nwords);         // [nwords + 1]
-  int32_t* ulist = wprefix + nwords + 1;                                  // [nb]
-  float* S = reinterpret_cast<float*>(ulist + nb);                        // [8][nb]
-  uintptr_t wp = reinterpret_cast<uintptr_t>(sm) + s2_head_bytes(D, nb) +
-                 static_cast<size_t>(kSelRows) * (nb > D ? nb : D) * 4;
-  wp = (wp + 15) & ~static_cast<uintptr_t>(15);
+  float* qsT = reinterpret_cast<float*>(sc_smem);                       // [D][8]
+  uint32_t* ubits = reinterpret_cast<uint32_t*>(qsT + kSelRows * D);    // [nwords]
+  uint32_t* rbits = ubits + nwords;                                     // [8][nwords]
+  int32_t* upre = reinterpret_cast<int32_t*>(rbits + kSelRows * nwords);  // [nwords]
+  int32_t* rpre = upre + nwords;                                        // [8][nwords]
+  uint32_t* nbits = reinterpret_cast<uint32_t*>(rpre + kSelRows * nwords);  // [8][nwords]
+  int32_t* ulist = reinterpret_cast<int32_t*>(nbits + kSelRows * nwords);  // [nb]
+  __shared__ int u_total;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint8_t* wbase = reinterpret_cast<uint8_t*>(wp) + static_cast<size_t>(warp) * sel_warp_bytes(cap);
-  uint32_t* bins32 = reinterpret_cast<uint32_t*>(wbase);   // [2][256]: low / high 18-bit sums
-  uint64_t* wgt = reinterpret_cast<uint64_t*>(wbase + 2048);
-  uint32_t* key = reinterpret_cast<uint32_t*>(wgt + cap);
-  uint8_t* flag = reinterpret_cast<uint8_t*>(key + cap);
-
-  const int I = I0 + warp;
-  const bool row_ok = I < nb;
+  const int bh = blockIdx.y;
+  const int I0 = blockIdx.x * kSelRows;
   const bool dynamic = p.mode == DYNRAD_DYNAMIC_THRESHOLD;
-  // Static mode without score export never needs the forced blocks' scores
-  // (they are kept regardless and k counts only the others).
+  // static mode without score export never needs the forced blocks' scores
   const bool skip_forced = !dynamic && p.scores_out == nullptr;
-  const int flo = row_ok ? p.forced_lo[I] : 0, fhi = row_ok ? p.forced_hi[I] : -1;
 
-  // 1. pooled queries of the 8 rows, transposed; clear the union bitmap
   for (int i = threadIdx.x; i < kSelRows * D; i += kS2Threads) {
     const int r = i / D, d = i % D;
     qsT[d * kSelRows + r] = (I0 + r < nb) ? p.qbar[(static_cast<int64_t>(bh) * nb + I0 + r) * D + d] : 0.f;
   }
-  for (int i = threadIdx.x; i < nwords; i += kS2Threads) bitmap[i] = 0u;
+  for (int i = threadIdx.x; i < kSelRows * nwords; i += kS2Threads) {
+    rbits[i] = 0u;
+    nbits[i] = 0u;
+  }
   __syncthreads();
-
-  // 2. union of the 8 candidate lists
+  // row bitmaps (warp r owns row I0 + r): every candidate (for ranks) and the
+  // candidates that need a score
+  const int I = I0 + warp;
   int c_beg = 0, n = 0;
-  if (row_ok) {
+  if (I < nb) {
     c_beg = p.cand_row_ptr[I];
     n = p.cand_row_ptr[I + 1] - c_beg;
-    if (n > cap || n < 0) {  // longer than the declared bound: the row stays empty
-      if (lane == 0) record_error(DYNRAD_ERR_CAPACITY);
-      n = 0;
-    }
-    for (int c = lane; c < n; c += 32) {
-      const int J = p.cand_col[c_beg + c];
-      if (!skip_forced || J < flo || J > fhi) atomicOr(&bitmap[J >> 5], 1u << (J & 31));
+    const int flo = p.forced_lo[I], fhi = p.forced_hi[I];
+    // the list is sorted, so lanes sharing a bitmap word are adjacent: OR their
+    // bits within the warp, one shared-memory update per word
+    for (int c0 = 0; c0 < n; c0 += 32) {
+      const int c = c0 + lane;
+      const bool in = c < n;
+      const int J = in ? p.cand_col[c_beg + c] : 0;
+      const int w = in ? (J >> 5) : -1 - lane;
+      const uint32_t bit = in ? 1u << (J & 31) : 0u;
+      const uint32_t need = (in && (!skip_forced || J < flo || J > fhi)) ? bit : 0u;
+      const unsigned grp = __match_any_sync(0xffffffffu, w);
+      const uint32_t all_bits = __reduce_or_sync(grp, bit);
+      const uint32_t need_bits = __reduce_or_sync(grp, need);
+      if (in && lane == __ffs(grp) - 1) {
+        rbits[warp * nwords + w] |= all_bits;
+        nbits[warp * nwords + w] |= need_bits;
+      }
+      __syncwarp();
     }
   }
   __syncthreads();
-
-  // 3. rank of every union member (word prefix popcounts) and the union list
-  if (warp == 0) {
+  // union bitmap
+  for (int w = threadIdx.x; w < nwords; w += kS2Threads) {
+    uint32_t u = 0;
+#pragma unroll
+    for (int r = 0; r < kSelRows; ++r) u |= nbits[r * nwords + w];
+    ubits[w] = u;
+  }
+  __syncthreads();
+  // prefix popcounts: warp r for row r; warp 0 also for the union
+  for (int which = warp; which <= kSelRows; which += kSelRows) {
+    const uint32_t* bits = which < kSelRows ? rbits + which * nwords : ubits;
+    int32_t* pre = which < kSelRows ? rpre + which * nwords : upre;
     int carry = 0;
     for (int w0 = 0; w0 < nwords; w0 += 32) {
       const int w = w0 + lane;
-      const int c = w < nwords ? __popc(bitmap[w]) : 0;
+      const int c = w < nwords ? __popc(bits[w]) : 0;
       int incl = c;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += y;
       }
-      if (w < nwords) wprefix[w] = carry + incl - c;
+      if (w < nwords) pre[w] = carry + incl - c;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) wprefix[nwords] = carry;
+    if (which == kSelRows && lane == 0) u_total = carry;
   }
   __syncthreads();
-  const int U = wprefix[nwords];
-  for (int w = threadIdx.x; w < nwords; w += kS2Threads) {
-    uint32_t bits = bitmap[w];
-    int pos = wprefix[w];
-    while (bits) {
-      const int b = __ffs(bits) - 1;
-      bits &= bits - 1;
-      ulist[pos++] = (w << 5) + b;
-    }
+  // union list, one word per warp iteration
+  for (int w = warp; w < nwords; w += kSelRows) {
+    const uint32_t bits = ubits[w];
+    if ((bits >> lane) & 1u) ulist[upre[w] + __popc(bits & ((1u << lane) - 1u))] = (w << 5) + lane;
   }
   __syncthreads();
-
-  // 4. block scores: thread handles union members u and u + 256; each kbar
-  //    value read (coalesced across consecutive members) feeds 8 rows
+  const int U = u_total;
   const float* kT = p.kbarT + static_cast<int64_t>(bh) * D * p.nbp;
+  float* out = p.scores + static_cast<int64_t>(bh) * p.cand_nnz;
   for (int u0 = threadIdx.x; u0 < U; u0 += 2 * kS2Threads) {
     const int u1 = u0 + kS2Threads;
     const int J0 = ulist[u0];
@@ -298,61 +315,114 @@ __device__ __forceinline__ void score_item(const Stage2Params& p, int bh, int I0
       a1[2] = __ffma2_rn(q45, kk1, a1[2]);
       a1[3] = __ffma2_rn(q67, kk1, a1[3]);
     }
+    // scatter to the rows that list each block
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      S[(2 * r) * nb + u0] = a0[r].x * p.scale;
-      S[(2 * r + 1) * nb + u0] = a0[r].y * p.scale;
-      if (u1 < U) {
-        S[(2 * r) * nb + u1] = a1[r].x * p.scale;
-        S[(2 * r + 1) * nb + u1] = a1[r].y * p.scale;
+    for (int e = 0; e < 2; ++e) {
+      if (e == 1 && u1 >= U) break;
+      const int J = e == 0 ? J0 : J1;
+      const int w = J >> 5;
+      const uint32_t below = (1u << (J & 31)) - 1u;
+#pragma unroll
+      for (int r = 0; r < kSelRows; ++r) {
+        const uint32_t bits = rbits[r * nwords + w];
+        if ((nbits[r * nwords + w] >> (J & 31)) & 1u) {
+          const float2 v = e == 0 ? a0[r >> 1] : a1[r >> 1];
+          const float sc = ((r & 1) ? v.y : v.x) * p.scale;
+          out[p.cand_row_ptr[I0 + r] + rpre[r * nwords + w] + __popc(bits & below)] = sc;
+        }
       }
     }
   }
-  __syncthreads();
-  if (!row_ok) return;
-  const int64_t bhl = bh;
-  if (n == 0) {
-    if (lane == 0) p.counts[bhl * nb + I] = 0;
+}
+
+// ---------------------------------------------------------------------------
+// Selection: one warp per query block; the row's candidates (block, score,
+// weight) live in registers, E per lane; a 2 x 256 x u32 bin array in shared
+// memory per warp holds the radix histograms.
+// ---------------------------------------------------------------------------
+constexpr int kSelWarps = 8;
+
+// DYN: dynamic-threshold mode (fp64 masses as fixed-point weights); otherwise
+// static-ratio mode, where every free block weighs 1 and only the keys are kept
+// in registers.
+template <int E, bool DYN>
+__global__ void __launch_bounds__(kSelWarps * 32, DYN ? (E <= 4 ? 4 : (E <= 8 ? 3 : (E <= 16 ? 2 : 1)))
+                                                      : (E <= 8 ? 4 : (E <= 16 ? 3 : 2)))
+    select_kernel(Stage2Params p) {
+  __shared__ uint32_t bins_all[kSelWarps][512];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* bins = bins_all[warp];
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kSelWarps + warp;
+  const int64_t rows = static_cast<int64_t>(p.nb) * p.rows_bh;
+  if (row >= rows) return;
+  const int64_t bh = row / p.nb;
+  const int I = static_cast<int>(row - bh * p.nb);
+  const int c_beg = p.cand_row_ptr[I];
+  int n = p.cand_row_ptr[I + 1] - c_beg;
+  if (n > 32 * E || n < 0) {  // longer than the declared bound: the row stays empty
+    if (lane == 0) {
+      record_error(DYNRAD_ERR_CAPACITY);
+      p.counts[row] = 0;
+    }
     return;
   }
-
-  // 5. selection for row I (one warp)
-  const int32_t* cols = p.cand_col + c_beg;
-  const float* Srow = S + warp * nb;
-  auto score_of = [&](int J) -> float {
-    const int w = J >> 5;
-    return Srow[wprefix[w] + __popc(bitmap[w] & ((1u << (J & 31)) - 1u))];
+  const int flo = p.forced_lo[I], fhi = p.forced_hi[I];
+  constexpr bool dynamic = DYN;
+  const float* srow = p.scores + bh * p.cand_nnz + c_beg;
+  int32_t Jv[DYN ? E : 1];
+  uint32_t key[E];
+  uint64_t wgt[DYN ? E : 1];
+  // weight of element i (static: 1 for every free block)
+  auto wof = [&](int i) -> uint64_t {
+    if constexpr (DYN) return wgt[i];
+    else return 1;
   };
+  uint32_t forced = 0, valid = 0;   // bit i: element i of this lane
   float smax = -INFINITY;
-  if (dynamic)
-    for (int c = lane; c < n; c += 32) smax = fmaxf(smax, score_of(cols[c]));
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, off));
+  for (int i = 0; i < E; ++i) {
+    const int c = lane + 32 * i;
+    if constexpr (DYN) {
+      Jv[i] = 0;
+      wgt[i] = 0;
+    }
+    key[i] = 0;
+    if (c < n) {
+      const int J = p.cand_col[c_beg + c];
+      const bool f = J >= flo && J <= fhi;
+      if constexpr (DYN) Jv[i] = J;
+      valid |= 1u << i;
+      forced |= (f ? 1u : 0u) << i;
+      const float sc = (f && !dynamic) ? 0.f : srow[c];
+      key[i] = order_key(sc);
+      if (dynamic) smax = fmaxf(smax, sc);
+    }
+  }
   uint64_t base = 0, ztot = 0;
   int nfree = 0;
-  for (int c0 = 0; c0 < n; c0 += 32) {
-    const int c = c0 + lane;
-    bool forced = false;
-    if (c < n) {
-      const int J = cols[c];
-      forced = J >= flo && J <= fhi;
-      const float s = (forced && skip_forced) ? 0.f : score_of(J);
-      if (p.scores_out != nullptr) p.scores_out[bhl * p.cand_nnz + c_beg + c] = s;
+  if (dynamic) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, off));
+  }
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    if ((valid >> i) & 1u) {
       uint64_t w = 1;
-      if (dynamic) {
-        const double e = exp(static_cast<double>(s) - static_cast<double>(smax));
+      if constexpr (DYN) {
+        const double e = exp(static_cast<double>(srow[lane + 32 * i]) - static_cast<double>(smax));
         w = __double2ull_rn(e * kMassScale);
+        wgt[i] = ((forced >> i) & 1u) ? 0 : w;
       }
-      wgt[c] = forced ? 0 : w;
-      key[c] = order_key(s);
-      flag[c] = forced ? 1 : 0;
-      if (forced) base += w;
+      if ((forced >> i) & 1u) base += w;
+      else ++nfree;
       ztot += w;
     }
-    nfree += __popc(__ballot_sync(0xffffffffu, c < n && !forced));
   }
   base = warp_sum_u64(base);
   ztot = warp_sum_u64(ztot);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) nfree += __shfl_xor_sync(0xffffffffu, nfree, off);
+  const uint32_t freev = valid & ~forced;
 
   Reach reach;
   reach.dynamic = dynamic;
@@ -363,37 +433,48 @@ __device__ __forceinline__ void score_item(const Stage2Params& p, int bh, int I0
   if (dynamic) {
     if (p.value >= 1.0) keep_all = true;
     else reach.tau_z = __dmul_rn(p.value, static_cast<double>(ztot));
-  } else {
-    if (nfree > 0) {
-      const double kf = floor(__dadd_rn(__dmul_rn(p.value, static_cast<double>(nfree)), 1e-9));
-      reach.k = kf < 1.0 ? 1ull : static_cast<uint64_t>(kf);
-      if (reach.k > static_cast<uint64_t>(nfree)) reach.k = nfree;
-    }
+  } else if (nfree > 0) {
+    const double kf = floor(__dadd_rn(__dmul_rn(p.value, static_cast<double>(nfree)), 1e-9));
+    reach.k = kf < 1.0 ? 1ull : static_cast<uint64_t>(kf);
+    if (reach.k > static_cast<uint64_t>(nfree)) reach.k = nfree;
   }
-  __syncwarp();
 
   uint32_t kstar = 0xFFFFFFFFu;  // cut key; free blocks with key > kstar are kept
   uint64_t above = 0;            // weight of free blocks with key > kstar
   const bool cut_none = !keep_all && reach(0);
   if (!keep_all && !cut_none) {
-    uint32_t prefix = 0, pmask = 0;
-    bool found = true;
-    for (int pass = 0; pass < 4 && found; ++pass) {
-      const int shift = 24 - 8 * pass;
+    // the free keys agree above their highest differing bit: start there
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) bins32[lane * 16 + i] = 0u;
+    for (int i = 0; i < E; ++i)
+      if ((freev >> i) & 1u) {
+        kmin = min(kmin, key[i]);
+        kmax = max(kmax, key[i]);
+      }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
+      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
+    }
+    const int top = (kmin == kmax) ? -1 : 31 - __clz(kmin ^ kmax);  // highest differing bit
+    uint32_t pmask = top >= 31 ? 0u : (0xFFFFFFFFu << (top + 1));
+    uint32_t prefix = kmax & pmask;
+    bool found = true;
+    for (int hi = top; hi >= 0 && found; hi -= 8) {
+      const int shift = hi >= 7 ? hi - 7 : 0;
+      const uint32_t dmask = (1u << (hi - shift + 1)) - 1u;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) bins[lane * 16 + i] = 0u;
       __syncwarp();
       // weights < 2^36 are split into 18-bit halves; each half's bin sum stays
-      // below 2^32 for rows of up to 2^14 candidates, so native 32-bit shared
-      // atomics give exact sums
-      for (int c = lane; c < n; c += 32) {
-        if (flag[c]) continue;
-        const uint32_t kk = key[c];
-        if ((kk & pmask) == prefix) {
-          const uint64_t w = wgt[c];
-          const uint32_t b = (kk >> shift) & 255u;
-          atomicAdd(&bins32[b], static_cast<uint32_t>(w & 0x3FFFFu));
-          if (w >> 18) atomicAdd(&bins32[256 + b], static_cast<uint32_t>(w >> 18));
+      // below 2^32 for rows of up to 2^14 candidates
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        if (((freev >> i) & 1u) && (key[i] & pmask) == prefix) {
+          const uint32_t b = (key[i] >> shift) & dmask;
+          const uint64_t w = wof(i);
+          atomicAdd(&bins[b], static_cast<uint32_t>(w & 0x3FFFFu));
+          if (w >> 18) atomicAdd(&bins[256 + b], static_cast<uint32_t>(w >> 18));
         }
       }
       __syncwarp();
@@ -402,7 +483,7 @@ __device__ __forceinline__ void score_item(const Stage2Params& p, int bh, int I0
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const uint32_t b = 255 - (lane * 8 + i);
-        loc[i] = (static_cast<uint64_t>(bins32[256 + b]) << 18) + bins32[b];
+        loc[i] = (static_cast<uint64_t>(bins[256 + b]) << 18) + bins[b];
         lsum += loc[i];
       }
       const uint64_t excl = warp_excl_scan_u64(lsum, lane);
@@ -429,60 +510,45 @@ __device__ __forceinline__ void score_item(const Stage2Params& p, int bh, int I0
       digit = __shfl_sync(0xffffffffu, digit, src);
       above = __shfl_sync(0xffffffffu, new_above, src);
       prefix |= digit << shift;
-      pmask |= 255u << shift;
+      pmask |= dmask << shift;
       __syncwarp();
     }
     if (found) kstar = prefix;
     else keep_all = true;  // target not reachable (rounding at tau ~ 1): keep all
   }
 
-  // 6. mark kept free blocks: key > kstar, and ties at kstar in ascending
-  //    order until the target is reached
+  // kept: forced, free with key > kstar, and ties at kstar in ascending order
+  // until the target is reached; written ascending
+  uint32_t kept = forced;
   if (!cut_none) {
     uint64_t tie_run = 0;
-    for (int c0 = 0; c0 < n; c0 += 32) {
-      const int c = c0 + lane;
-      bool kept = false;
-      if (c < n && !flag[c] && (keep_all || key[c] > kstar)) kept = true;
-      const bool tie = !keep_all && c < n && !flag[c] && key[c] == kstar;
-      const uint64_t tw = tie ? wgt[c] : 0;
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const bool fr = (freev >> i) & 1u;
+      bool k_ = fr && (keep_all || key[i] > kstar);
+      const bool tie = !keep_all && fr && key[i] == kstar;
+      const uint64_t tw = tie ? wof(i) : 0;
       const uint64_t ex = warp_excl_scan_u64(tw, lane);
-      if (tie && !reach(above + tie_run + ex)) kept = true;
+      if (tie && !reach(above + tie_run + ex)) k_ = true;
       tie_run += warp_sum_u64(tw);
-      if (c < n && kept) flag[c] = 1;
+      kept |= (k_ ? 1u : 0u) << i;
     }
   }
-  __syncwarp();
-
-  // 7. ordered output of the kept blocks
-  int32_t* dst = p.kept_tmp + bhl * p.cand_nnz + c_beg;
+  int32_t* dst = p.kept_tmp + bh * p.cand_nnz + c_beg;
   int cnt = 0;
-  for (int c0 = 0; c0 < n; c0 += 32) {
-    const int c = c0 + lane;
-    const bool k_ = c < n && flag[c];
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    const bool k_ = (kept >> i) & 1u;
     const unsigned bal = __ballot_sync(0xffffffffu, k_);
-    if (k_) dst[cnt + __popc(bal & ((1u << lane) - 1u))] = cols[c];
+    if (k_) {
+      int32_t J;
+      if constexpr (DYN) J = Jv[i];
+      else J = p.cand_col[c_beg + lane + 32 * i];
+      dst[cnt + __popc(bal & ((1u << lane) - 1u))] = J;
+    }
     cnt += __popc(bal);
   }
-  if (lane == 0) p.counts[bhl * nb + I] = cnt;
-}
-
-// Pool: one CTA per (tensor, head, 8 consecutive blocks); many CTAs per SM keep
-// enough loads in flight to run at HBM bandwidth.
-template <int D>
-__global__ void __launch_bounds__(kS2Threads, 4) pool_kernel(Stage2Params p) {
-  __shared__ __align__(16) float tile[kSelRows * D];
-  const int nq = (p.nb + kSelRows - 1) / kSelRows;
-  const int grp = blockIdx.x % nq;
-  const bool is_k = (blockIdx.x / nq) != 0;
-  pool_item<D>(p, is_k, blockIdx.y, grp, tile);
-}
-
-// Score + select: one CTA per (head, 8 consecutive query blocks).
-template <int D>
-__global__ void __launch_bounds__(kS2Threads, 2) select_kernel(Stage2Params p) {
-  extern __shared__ __align__(16) uint8_t s2_smem[];
-  score_item<D>(p, blockIdx.y, blockIdx.x * kSelRows, s2_smem);
+  if (lane == 0) p.counts[row] = cnt;
 }
 
 // ---------------------------------------------------------------------------

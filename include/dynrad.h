@@ -132,8 +132,10 @@ size_t dynrad_select_workspace_bytes(int32_t B, int32_t H, int32_t N, int32_t D,
  *   D             64 or 128
  *   cand_*, forced_*   stage-1 output for the same geometry; cand_nnz its total
  *   cand_max_row  longest candidate row (stage 1's max_row_out), or 0 for the
- *                 bound Nb; it sizes shared memory.  A row longer than this is
- *                 an error (device status DYNRAD_ERR_CAPACITY, row left empty)
+ *                 bound Nb; it sizes the selection's per-warp register arrays.
+ *                 Rows of up to 1024 candidates are supported (a larger bound
+ *                 returns DYNRAD_ERR_UNSUPPORTED); a row longer than the bound
+ *                 is an error (device status DYNRAD_ERR_CAPACITY, row left empty)
  *   row_ptr       device int32 [B*H*Nb + 1]; row (b*H + h)*Nb + I
  *   col_idx       device int32 [col_cap]; col_cap >= B*H*cand_nnz always suffices
  *   scores_out    device fp32 [B*H*cand_nnz] or NULL: the fp32 scores in
