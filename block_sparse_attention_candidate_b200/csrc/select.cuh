@@ -1,5 +1,5 @@
 // Stage 2: block pooling, block proxy scores and the two selection modes
-// (DynamicRad, Sec. 3.2 and Algorithm 1 lines 15-22, in block-pooled form).
+// (DynamicRad, Sec. 3.2 and Algorithm 1, selection steps, in block-pooled form).
 //
 // Two launches:
 //

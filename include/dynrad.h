@@ -6,7 +6,7 @@
  * Long Video Diffusion" (arXiv 2604.20470).  Three stages:
  *
  *   1. dynrad_build_candidates -- the radial candidate block set of Sec. 3.1
- *      (Eqs. 1-7, "Density control within blocks"; Algorithm 1 lines 4-14, 23).
+ *      (Eqs. 1-7, "Density control within blocks"; Algorithm 1, candidate construction and block aggregation).
  *   2. dynrad_select_blocks    -- per query block, mean-pooled block scores
  *      (the 1/sqrt(d) logit scale of Eq. 9) and one of the two selection modes
  *      of Sec. 3.2: static-ratio (top rho fraction, k rule of Eq. 8) or
@@ -113,8 +113,8 @@ size_t dynrad_select_workspace_bytes(int32_t B, int32_t H, int32_t N, int32_t D,
                                      const dynrad_geom *geom, int64_t cand_nnz);
 
 /*
- * Stage 2: block pooling, scoring and selection (Sec. 3.2, Algorithm 1 lines
- * 15-22, in the block-pooled form).
+ * Stage 2: block pooling, scoring and selection (Sec. 3.2, the selection
+ * steps of Algorithm 1, in the block-pooled form).
  *
  * For every (b, h) and query block I: qbar_I, kbar_J = fp32 means of Q and K
  * over the valid tokens of each block; s_IJ = qbar_I . kbar_J * (1/sqrt(D))

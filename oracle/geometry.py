@@ -1,4 +1,5 @@
-"""Radial candidate block set (DynamicRad, Sec. 3.1, Eqs. 1-7; Algorithm 1 steps 4-14, 23).
+"""Radial candidate block set (DynamicRad, Sec. 3.1, Eqs. 1-7; Algorithm 1, candidate
+construction and block aggregation).
 
 Test infrastructure only (see the package docstring).
 
@@ -11,7 +12,7 @@ Readings where the paper is silent or loose:
   distance is |u - v| exactly as Eq. 7 writes it.
 * The rounding bracket of Eq. 3 is round-half-up, floor(x + 0.5).
 * Eq. 5's epsilon is a parameter (default 1e-6).
-* t = 0 pairs are always retained with w = N_t (Eq. 3 and Algorithm 1 line 6-8);
+* t = 0 pairs are always retained with w = N_t (Eq. 3 and Algorithm 1, intra-frame case);
   Eq. 6's split rule applies to t >= 1.
 * "Density control": a key token (column) of block J is active for query block I
   when the number of tokens of I linked to it exceeds theta_c * n_I; J is a
