@@ -246,6 +246,8 @@ def main():
     ap.add_argument("--workload", default="wan14b_720p", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-chunk", type=int, default=4,
+                    help="(batch, head) rows per chunk of the end-to-end host path")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=12, help="query blocks per run in the CPU sample")
     ap.add_argument("--ref-rows", type=int, default=3, help="query blocks per run per reference step")
@@ -404,23 +406,26 @@ def main():
                  "speedup_vs_dense": {lbl: round(dense_ms / ri["attn_ms"], 2) for lbl, ri in run_info.items()}}
         del rp, col, o, lse
 
-    # ---- end to end: pinned host inputs -> device -> path -> outputs back
+    # ---- end to end through the host-memory entry point: pinned host Q, K, V
+    # in, every run's O and LSE back to pinned host memory, the copies
+    # overlapped with the kernels by dynrad_host_path (chunks of heads)
     e2e = None
     if not args.no_e2e:
-        out_host_o = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
-        out_host_l = torch.empty((B, H, N), dtype=torch.float32, pin_memory=True)
-        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        h2d = 3 * q.numel() * 2
-        d2h = len(runs) * (q.numel() * 2 + B * H * N * 4)
+        del q, k, v
+        for r in runs:
+            del r["o"], r["lse"]
+        torch.cuda.empty_cache()
+        hruns = [{"geom": r["geom"], "cand": r["cand"], "mode": r["mode"], "value": r["value"],
+                  "o_host": torch.empty((B, H, N, D), dtype=torch.bfloat16, pin_memory=True),
+                  "lse_host": torch.empty((B, H, N), dtype=torch.float32, pin_memory=True)} for r in runs]
+        hws = abi.HostPathWorkspace(B, H, N, D, hruns, args.e2e_chunk, dev)
+        h2d = 3 * B * H * N * D * 2
+        d2h = len(runs) * (B * H * N * D * 2 + B * H * N * 4)
 
         def e2e_step():
-            qd.copy_(host["q"], non_blocking=True)
-            kd.copy_(host["k"], non_blocking=True)
-            vd.copy_(host["v"], non_blocking=True)
             for r in runs:
-                run_path(r, qd, kd, vd)
-                out_host_o.copy_(r["o"], non_blocking=True)
-                out_host_l.copy_(r["lse"], non_blocking=True)
+                abi.dynrad_build_candidates_into(r["geom"], r["cand"])
+            abi.dynrad_host_path(host["q"], host["k"], host["v"], hruns, chunk_bh=args.e2e_chunk, workspace=hws)
 
         for _ in range(2):
             e2e_step()
@@ -434,10 +439,14 @@ def main():
             e2e_step()
         a1.record(stream)
         torch.cuda.synchronize()
+        st = abi.dynrad_device_status(clear=True)
+        if st != 0:
+            raise RuntimeError(f"device status after the end-to-end run: {abi.status_string(st)}")
         e2e_ms = max_over_ranks(a0.elapsed_time(a1), dev)
         e2e = {"value": world * flops_step * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": e2e_ms / args.steps}
+               "ms_per_step": e2e_ms / args.steps,
+               "path": f"dynrad_host_path, pinned host buffers, chunks of {args.e2e_chunk} heads"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

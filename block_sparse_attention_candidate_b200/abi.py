@@ -39,6 +39,8 @@ EXPORTED = (
     "dynrad_debug_exp2",
     "dynrad_static_scratch_bytes",
     "dynrad_select_blocks_static_scratch",
+    "dynrad_host_path_workspace_bytes",
+    "dynrad_host_path",
 )
 
 
@@ -54,6 +56,22 @@ class DynradGeom(ctypes.Structure):
         ("theta_m", ctypes.c_double),
         ("eps", ctypes.c_double),
         ("force_t", ctypes.c_int32),
+    ]
+
+
+class DynradHostRun(ctypes.Structure):
+    _fields_ = [
+        ("geom", DynradGeom),
+        ("cand_row_ptr", ctypes.c_void_p),
+        ("cand_col", ctypes.c_void_p),
+        ("cand_nnz", ctypes.c_int64),
+        ("cand_max_row", ctypes.c_int64),
+        ("forced_lo", ctypes.c_void_p),
+        ("forced_hi", ctypes.c_void_p),
+        ("mode", ctypes.c_int32),
+        ("rho_or_tau", ctypes.c_double),
+        ("o_host", ctypes.c_void_p),
+        ("lse_host", ctypes.c_void_p),
     ]
 
 
@@ -108,6 +126,12 @@ def lib() -> ctypes.CDLL:
         L.dynrad_select_blocks_static_scratch.argtypes = [_VP, _VP, _I32, _I32, _I32, _I32, _GP, _VP, _VP, _I64,
                                                           _I64, _VP, _VP, _I32, ctypes.c_double, _VP, _VP, _I64,
                                                           _VP, _VP]
+        L.dynrad_host_path_workspace_bytes.restype = _SZ
+        L.dynrad_host_path_workspace_bytes.argtypes = [_I32, _I32, _I32, _I32, ctypes.POINTER(DynradHostRun), _I32,
+                                                       _I32]
+        L.dynrad_host_path.restype = ctypes.c_int
+        L.dynrad_host_path.argtypes = [_VP, _VP, _VP, _I32, _I32, _I32, _I32, ctypes.POINTER(DynradHostRun), _I32,
+                                       _I32, ctypes.c_float, _VP, _SZ, _VP]
         _lib = L
     return _lib
 
@@ -267,3 +291,55 @@ def dynrad_device_status(clear: bool = True, stream=None) -> int:
     _check(lib().dynrad_device_status(ctypes.byref(v), 1 if clear else 0, _stream(stream)),
            "dynrad_device_status")
     return int(v.value)
+
+
+def make_host_runs(runs) -> ctypes.Array:
+    """C array of dynrad_host_run from dicts with geom, cand (from
+    dynrad_build_candidates), mode, value, o_host, lse_host (pinned CPU
+    tensors bf16 [B, H, N, D] / fp32 [B, H, N])."""
+    arr = (DynradHostRun * len(runs))()
+    for i, r in enumerate(runs):
+        c = r["cand"]
+        for t in (r["o_host"], r["lse_host"]):
+            if t.is_cuda or not t.is_contiguous():
+                raise ValueError("o_host / lse_host must be contiguous host tensors")
+        arr[i] = DynradHostRun(make_geom(r["geom"]), c["row_ptr"].data_ptr(), c["col"].data_ptr(), c["nnz"],
+                               c["max_row"], c["forced_lo"].data_ptr(), c["forced_hi"].data_ptr(),
+                               MODES[r["mode"]] if isinstance(r["mode"], str) else int(r["mode"]), float(r["value"]),
+                               r["o_host"].data_ptr(), r["lse_host"].data_ptr())
+    return arr
+
+
+def dynrad_host_path_workspace_bytes(B, H, N, D, runs, chunk_bh) -> int:
+    arr = make_host_runs(runs)
+    return int(lib().dynrad_host_path_workspace_bytes(B, H, N, D, arr, len(runs), int(chunk_bh)))
+
+
+class HostPathWorkspace:
+    """Device workspace of dynrad_host_path (reusable across calls)."""
+
+    def __init__(self, B, H, N, D, runs, chunk_bh, device=None):
+        device = device or torch.device("cuda", torch.cuda.current_device())
+        n = dynrad_host_path_workspace_bytes(B, H, N, D, runs, chunk_bh)
+        if n == 0:
+            raise DynradError(DYNRAD_ERR_INVALID_ARG, "dynrad_host_path_workspace_bytes")
+        self.buffer = torch.empty(n + 256, dtype=torch.uint8, device=device)
+        off = (-self.buffer.data_ptr()) % 256
+        self.view = self.buffer[off:off + n]
+
+
+def dynrad_host_path(q_host, k_host, v_host, runs, chunk_bh=4, scale=0.0, workspace=None, stream=None):
+    """Stages 2 and 3 from pinned host Q, K, V (bf16 [B, H, N, D]) to each
+    run's pinned host o_host / lse_host, copies overlapped with the kernels.
+    Asynchronous on `stream` (torch's current stream by default)."""
+    for t in (q_host, k_host, v_host):
+        if t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError("q_host, k_host, v_host must be contiguous bf16 host tensors")
+    B, H, N, D = q_host.shape
+    arr = make_host_runs(runs)
+    ws = workspace or HostPathWorkspace(B, H, N, D, runs, chunk_bh)
+    _check(lib().dynrad_host_path(ctypes.c_void_p(q_host.data_ptr()), ctypes.c_void_p(k_host.data_ptr()),
+                                  ctypes.c_void_p(v_host.data_ptr()), B, H, N, D, arr, len(runs), int(chunk_bh),
+                                  float(scale), _ptr(ws.view), ws.view.numel(), _stream(stream)),
+           "dynrad_host_path")
+    return ws

@@ -14,7 +14,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libdynrad.so")
-SOURCES = ["dynrad.cu"]
+SOURCES = ["dynrad.cu", "host_path.cu"]
 HEADERS = ["common.cuh", "candidates.cuh", "select.cuh", "attention.cuh"]
 
 

@@ -27,7 +27,8 @@
  *     attended, padded query rows are never written).  Nb = ceil(N / block).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) unless stated.  The library allocates no memory and frees none of
- *     the caller's.
+ *     the caller's (dynrad_host_path creates, and releases, two streams and a
+ *     few events per call).
  *   - Every call returns a dynrad_status.  Argument errors are found on the
  *     host before any launch.  Errors found by a kernel (capacity exceeded, a
  *     bounded wait that ran out) are recorded in a device status word read by
@@ -209,6 +210,73 @@ int dynrad_sparse_attn(const void *q, const void *k, const void *v, int32_t B,
                        const int32_t *row_ptr, const int32_t *col_idx,
                        float scale, void *o, float *lse,
                        dynrad_stream_t stream);
+
+/*
+ * Stages 2 and 3 from and to HOST memory (no counterpart in the paper: a
+ * runtime convenience for callers whose Q, K, V live on the host).
+ *
+ * For each of n_runs selection settings ("runs": geometry, candidate set,
+ * mode, rho or tau) over one layer's Q, K, V, computes the kept-block CSR
+ * (as dynrad_select_blocks) and the attention output (as dynrad_sparse_attn)
+ * and writes the run's O and LSE to host memory.  The B*H (batch, head) rows
+ * go through in chunks of chunk_bh rows: the copy-in of later chunks, the
+ * kernels of the current chunk and the copy-out of finished (chunk, run)
+ * outputs run concurrently on two streams the call creates and on `stream`.
+ * Results are bit-identical to the device-resident calls (every stage is
+ * independent per (batch, head) row).
+ *
+ *   q_host, k_host, v_host  HOST bf16 [B, H, N, D]; pinned (page-locked)
+ *                 memory for the copies to overlap (pageable memory works but
+ *                 serialises)
+ *   runs[r].geom, cand_*, forced_*  as for dynrad_select_blocks (candidate
+ *                 CSR from dynrad_build_candidates for that geometry; DEVICE)
+ *   runs[r].mode, rho_or_tau  as for dynrad_select_blocks
+ *   runs[r].o_host, lse_host  HOST bf16 [B, H, N, D] and fp32 [B, H, N]
+ *                 (pinned for overlap)
+ *   n_runs        1 .. 16
+ *   chunk_bh      rows per chunk (>= 1; the last chunk may be shorter).
+ *                 Chunks of a whole number of waves of the attention kernel
+ *                 keep it efficient (e.g. 4 heads of 75,600 tokens = 1,184
+ *                 CTAs = 8 x 148 SMs).
+ *   scale         as for dynrad_sparse_attn (0 means 1/sqrt(D))
+ *   workspace     DEVICE, 256-byte aligned, at least
+ *                 dynrad_host_path_workspace_bytes(...) bytes: it holds Q, K, V,
+ *                 every run's O and LSE, and one chunk's kept CSR and
+ *                 selection workspace
+ *
+ * Ordering: the call's device work starts after the work already queued on
+ * `stream` and `stream` continues only after the last copy-out, so back-to-
+ * back calls on one stream never overlap.  The host buffers must stay valid
+ * and unchanged until `stream` has passed the call.
+ * Errors: DYNRAD_ERR_INVALID_ARG (null pointer, n_runs or chunk_bh out of
+ * range, a geometry that does not match N, misaligned workspace),
+ * DYNRAD_ERR_CAPACITY (workspace too small) -- both before any device work;
+ * otherwise the errors of dynrad_select_blocks / dynrad_sparse_attn, and
+ * DYNRAD_ERR_CUDA when a copy, stream or event call fails.
+ * dynrad_host_path_workspace_bytes returns 0 for arguments it cannot size.
+ */
+typedef struct dynrad_host_run {
+  dynrad_geom geom;
+  const int32_t *cand_row_ptr;
+  const int32_t *cand_col;
+  int64_t cand_nnz;
+  int64_t cand_max_row;
+  const int32_t *forced_lo;
+  const int32_t *forced_hi;
+  int32_t mode;
+  double rho_or_tau;
+  void *o_host;
+  float *lse_host;
+} dynrad_host_run;
+
+size_t dynrad_host_path_workspace_bytes(int32_t B, int32_t H, int32_t N,
+                                        int32_t D, const dynrad_host_run *runs,
+                                        int32_t n_runs, int32_t chunk_bh);
+int dynrad_host_path(const void *q_host, const void *k_host,
+                     const void *v_host, int32_t B, int32_t H, int32_t N,
+                     int32_t D, const dynrad_host_run *runs, int32_t n_runs,
+                     int32_t chunk_bh, float scale, void *workspace,
+                     size_t workspace_bytes, dynrad_stream_t stream);
 
 /*
  * Reads the device status word (the first error a kernel recorded since the

@@ -114,3 +114,75 @@ def test_workspace_size_formula():
     # kept lists + scan partials, each 256-byte aligned
     need = rows * 128 * 4 + 40 * 128 * nbp * 4 + 40 * nnz * 4
     assert need <= ws < need + 4096
+
+
+def _c_layout(struct, fields):
+    """sizeof / offsetof of a struct of include/dynrad.h, from gcc."""
+    import shutil
+    import subprocess
+    import tempfile
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    body = "\n".join(f'  printf("%zu\\n", offsetof({struct}, {f}));' for f in fields)
+    src = (f'#include <stddef.h>\n#include <stdio.h>\n#include "dynrad.h"\n'
+           f'int main(void) {{\n  printf("%zu\\n", sizeof({struct}));\n{body}\n  return 0;\n}}\n')
+    with tempfile.TemporaryDirectory() as d:
+        c, exe = os.path.join(d, "l.c"), os.path.join(d, "l")
+        open(c, "w").write(src)
+        subprocess.run(["gcc", "-I", os.path.dirname(HEADER), "-o", exe, c], check=True)
+        out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout.split()
+    return [int(x) for x in out]
+
+
+def test_host_run_struct_layout_matches_c():
+    names = [f[0] for f in abi.DynradHostRun._fields_]
+    got = _c_layout("dynrad_host_run", names)
+    assert got[0] == ctypes.sizeof(abi.DynradHostRun)
+    for n, off in zip(names, got[1:]):
+        assert getattr(abi.DynradHostRun, n).offset == off, n
+
+
+def _fake_runs(n, geom, o=0x20000, nnz=100):
+    arr = (abi.DynradHostRun * max(1, n))()
+    for i in range(n):
+        arr[i] = abi.DynradHostRun(abi.make_geom(geom), 0x10000, 0x10000, nnz, 0, 0x10000, 0x10000, 0, 0.25,
+                                   o, 0x30000)
+    return arr
+
+
+def test_host_path_argument_errors_before_any_device_work():
+    L = abi.lib()
+    geom = WORKLOADS["tiny"].geom
+    n = geom.n_tokens
+    p = ctypes.c_void_p(0x10000)
+    ws = ctypes.c_void_p(0x100000)   # 256-byte aligned, never dereferenced on these paths
+
+    def call(runs=None, n_runs=2, chunk=1, ws_ptr=ws, ws_bytes=1 << 40, q=p, N=n, D=64, scale=0.0):
+        runs = _fake_runs(2, geom) if runs is None else runs
+        return L.dynrad_host_path(q, p, p, 1, 2, N, D, runs, n_runs, chunk, scale, ws_ptr, ws_bytes, None)
+
+    assert call(q=None) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(n_runs=0) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(runs=_fake_runs(17, geom), n_runs=17) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(chunk=0) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(N=n + 1) == abi.DYNRAD_ERR_INVALID_ARG            # geometry does not match N
+    assert call(D=96) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(ws_ptr=ctypes.c_void_p(0x100010)) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(ws_bytes=4096) == abi.DYNRAD_ERR_CAPACITY
+    assert call(runs=_fake_runs(2, geom, o=0)) == abi.DYNRAD_ERR_INVALID_ARG   # null o_host
+    assert call(scale=-1.0) == abi.DYNRAD_ERR_INVALID_ARG
+    assert L.dynrad_host_path_workspace_bytes(1, 2, n, 64, _fake_runs(2, geom), 0, 1) == 0
+
+
+def test_host_path_workspace_size_formula():
+    L = abi.lib()
+    wl = WORKLOADS["wan14b_720p"]
+    g = wl.geom
+    B, H, N, D, chunk, nnz = 1, 40, g.n_tokens, 128, 4, 331078
+    runs = _fake_runs(4, g, nnz=nnz)
+    got = L.dynrad_host_path_workspace_bytes(B, H, N, D, runs, 4, chunk)
+    qkv = B * H * N * D * 2
+    sel = abi.dynrad_select_workspace_bytes(1, chunk, N, D, g, nnz)
+    # Q, K, V; O and LSE per run; one chunk's kept CSR and selection workspace
+    need = 3 * qkv + 4 * (qkv + B * H * N * 4) + (chunk * g.n_blocks + 1) * 4 + chunk * nnz * 4 + sel
+    assert need <= got < need + 256 * 16
