@@ -8,7 +8,8 @@
 // as soon as its inputs are in, and a copy-out stream returns each (chunk, run)
 // O and LSE as soon as its attention kernel is done.  PCIe is full duplex, so
 // with enough chunks the copies hide behind the kernels except for the first
-// chunk's copy-in and the last chunk's copy-out.
+// chunk's copy-in and the last chunk's copy-out, which the schedule keeps small
+// (chunks of 1 and 2 rows at both ends).
 //
 // Every stage is independent per (batch, head) row (the candidate set is
 // shared geometry, the selection and the attention never mix rows), so a
@@ -19,6 +20,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <utility>
 #include <vector>
 
 #include "dynrad.h"
@@ -136,7 +138,26 @@ int dynrad_host_path(const void* q_host, const void* k_host, const void* v_host,
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const int64_t bh = static_cast<int64_t>(B) * H;
   const int64_t chunk = std::min<int64_t>(chunk_bh, bh);
-  const int64_t n_chunks = (bh + chunk - 1) / chunk;
+  // Chunk schedule: (first row, rows).  Only the first chunk's copy-in and the
+  // last chunk's copy-out are not hidden behind kernels, so with room for it
+  // the schedule starts and ends with chunks of 1 and 2 rows.
+  std::vector<std::pair<int64_t, int64_t>> sched;
+  {
+    const bool ramp = chunk >= 4 && bh >= 2 * chunk + 6;
+    int64_t r = 0;
+    const int64_t edge[2] = {1, 2};
+    if (ramp)
+      for (int64_t e : edge) sched.push_back({r, e}), r += e;
+    const int64_t mid_end = ramp ? bh - 3 : bh;
+    while (r < mid_end) {
+      const int64_t n = std::min(chunk, mid_end - r);
+      sched.push_back({r, n});
+      r += n;
+    }
+    if (ramp)
+      for (int i = 1; i >= 0; --i) sched.push_back({r, edge[i]}), r += edge[i];
+  }
+  const int64_t n_chunks = static_cast<int64_t>(sched.size());
   const size_t row_in = static_cast<size_t>(N) * D * 2;   // bytes of one row of Q, K, V or O
   const size_t row_lse = static_cast<size_t>(N) * 4;
 
@@ -156,7 +177,7 @@ int dynrad_host_path(const void* q_host, const void* k_host, const void* v_host,
   const void* src[3] = {q_host, k_host, v_host};
   const size_t dst[3] = {L.q, L.k, L.v};
   for (int64_t c = 0; c < n_chunks; ++c) {
-    const int64_t r0 = c * chunk, rows = std::min(chunk, bh - r0);
+    const int64_t r0 = sched[c].first, rows = sched[c].second;
     for (int t = 0; t < 3; ++t) {
       if (cudaMemcpyAsync(ws + dst[t] + r0 * row_in, static_cast<const uint8_t*>(src[t]) + r0 * row_in,
                           rows * row_in, cudaMemcpyHostToDevice, co.in) != cudaSuccess)
@@ -170,7 +191,7 @@ int dynrad_host_path(const void* q_host, const void* k_host, const void* v_host,
   int32_t* row_ptr = reinterpret_cast<int32_t*>(ws + L.row_ptr);
   int32_t* col = reinterpret_cast<int32_t*>(ws + L.col);
   for (int64_t c = 0; c < n_chunks; ++c) {
-    const int64_t r0 = c * chunk, rows = std::min(chunk, bh - r0);
+    const int64_t r0 = sched[c].first, rows = sched[c].second;
     if (cudaStreamWaitEvent(main, in_done[c], 0) != cudaSuccess) return DYNRAD_ERR_CUDA;
     const uint8_t* qc = ws + L.q + r0 * row_in;
     const uint8_t* kc = ws + L.k + r0 * row_in;

@@ -234,7 +234,9 @@ int dynrad_sparse_attn(const void *q, const void *k, const void *v, int32_t B,
  *   runs[r].o_host, lse_host  HOST bf16 [B, H, N, D] and fp32 [B, H, N]
  *                 (pinned for overlap)
  *   n_runs        1 .. 16
- *   chunk_bh      rows per chunk (>= 1; the last chunk may be shorter).
+ *   chunk_bh      rows per chunk (>= 1; the last chunk may be shorter; with
+ *                 room for it, chunks of 1 and 2 rows open and close the
+ *                 schedule to shorten the copies that cannot overlap).
  *                 Chunks of a whole number of waves of the attention kernel
  *                 keep it efficient (e.g. 4 heads of 75,600 tokens = 1,184
  *                 CTAs = 8 x 148 SMs).
