@@ -69,7 +69,7 @@ int check_geom(const dynrad_geom* g, GeomDev* out) {
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct SelectWorkspace {
-  size_t qbar, kbar, kept, partial, total;
+  size_t qbar, kbar, kept, partial, plan_off, plan_cnt, plan_alloc, plan_J, plan_pos, total;
 };
 
 SelectWorkspace select_layout(int64_t bh, int64_t nb, int64_t d, int64_t cand_nnz) {
@@ -80,7 +80,15 @@ SelectWorkspace select_layout(int64_t bh, int64_t nb, int64_t d, int64_t cand_nn
   w.kbar = align256(w.qbar + static_cast<size_t>(rows * d) * 4);
   w.kept = align256(w.kbar + static_cast<size_t>(bh * d * padded_blocks(static_cast<int>(nb))) * 4);
   w.partial = align256(w.kept + static_cast<size_t>(bh * cand_nnz) * 4);
-  w.total = align256(w.partial + static_cast<size_t>(tiles) * 8);
+  // scoring plan: per group of 8 rows, the union list and the scatter positions
+  // (independent of the head; the unions' total is at most cand_nnz)
+  const int64_t groups = (nb + kSelRows - 1) / kSelRows;
+  w.plan_off = align256(w.partial + static_cast<size_t>(tiles) * 8);
+  w.plan_cnt = align256(w.plan_off + static_cast<size_t>(groups) * 4);
+  w.plan_alloc = align256(w.plan_cnt + static_cast<size_t>(groups) * 4);
+  w.plan_J = align256(w.plan_alloc + 4);
+  w.plan_pos = align256(w.plan_J + static_cast<size_t>(cand_nnz) * 4);
+  w.total = align256(w.plan_pos + static_cast<size_t>(cand_nnz) * kSelRows * 4);
   return w;
 }
 
@@ -312,6 +320,11 @@ int dynrad_select_blocks(const void* q, const void* k, int32_t B, int32_t H, int
     // and then, row by row, the kept lists (a row's warp reads all its scores
     // before it writes)
     sp.scores = scores_out != nullptr ? scores_out : reinterpret_cast<float*>(kept);
+    sp.plan_off = reinterpret_cast<int32_t*>(ws + w.plan_off);
+    sp.plan_cnt = reinterpret_cast<int32_t*>(ws + w.plan_cnt);
+    sp.plan_alloc = reinterpret_cast<int32_t*>(ws + w.plan_alloc);
+    sp.plan_J = reinterpret_cast<int32_t*>(ws + w.plan_J);
+    sp.plan_pos = reinterpret_cast<int32_t*>(ws + w.plan_pos);
     sp.rows_bh = static_cast<int>(bh);
     sp.cand_nnz = cand_nnz;
     sp.N = N;
@@ -324,25 +337,27 @@ int dynrad_select_blocks(const void* q, const void* k, int32_t B, int32_t H, int
     sp.value = rho_or_tau;
     sp.scale = 1.0f / std::sqrt(static_cast<float>(D));
     const int nq = (g.nb + kSelRows - 1) / kSelRows;
+    // scoring plan (candidate CSR only, shared by all heads)
+    const size_t psmem = plan_smem_bytes(g.nb);
+    if (psmem > 227 * 1024) return DYNRAD_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(psmem)) !=
+        cudaSuccess)
+      return DYNRAD_ERR_CUDA;
+    if (cudaMemsetAsync(sp.plan_alloc, 0, 4, st) != cudaSuccess) return DYNRAD_ERR_CUDA;
+    plan_kernel<<<nq, kS2Threads, psmem, st>>>(sp);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
     const dim3 pgrid(2 * nq, static_cast<unsigned>(bh));
     if (D == 128)
       pool_kernel<128><<<pgrid, kS2Threads, 0, st>>>(sp);
     else
       pool_kernel<64><<<pgrid, kS2Threads, 0, st>>>(sp);
     if ((rc = launch_status()) != DYNRAD_OK) return rc;
-    // scoring: union of 8 rows per CTA, scores to their candidate positions
-    const size_t ssmem = score_smem_bytes(D, g.nb);
-    if (ssmem > 227 * 1024) return DYNRAD_ERR_UNSUPPORTED;
-    const void* skern = D == 128 ? reinterpret_cast<const void*>(score_kernel<128>)
-                                 : reinterpret_cast<const void*>(score_kernel<64>);
-    if (cudaFuncSetAttribute(skern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ssmem)) !=
-        cudaSuccess)
-      return DYNRAD_ERR_CUDA;
+    // scoring: one CTA per (group of 8 rows, head), scores to their positions
     const dim3 sgrid(nq, static_cast<unsigned>(bh));
     if (D == 128)
-      score_kernel<128><<<sgrid, kS2Threads, ssmem, st>>>(sp);
+      score_kernel<128><<<sgrid, kS2Threads, 0, st>>>(sp);
     else
-      score_kernel<64><<<sgrid, kS2Threads, ssmem, st>>>(sp);
+      score_kernel<64><<<sgrid, kS2Threads, 0, st>>>(sp);
     if ((rc = launch_status()) != DYNRAD_OK) return rc;
     // selection: one warp per row, candidates in registers
     const unsigned rblocks = static_cast<unsigned>((rows + kSelWarps - 1) / kSelWarps);

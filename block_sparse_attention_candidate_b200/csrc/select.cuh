@@ -67,6 +67,11 @@ struct Stage2Params {
   int32_t* kept_tmp;        // [BH, cand_nnz] kept lists at the candidate offsets
   float* scores_out;        // nullable (caller's export of the scores)
   float* scores;            // [BH, cand_nnz] scores used by the selection
+  int32_t* plan_off;        // [groups] first plan entry of each group of 8 rows
+  int32_t* plan_cnt;        // [groups] union size of each group
+  int32_t* plan_alloc;      // [1] plan entries handed out (zeroed before the plan kernel)
+  int32_t* plan_J;          // [cand_nnz] union members (key blocks), per group ascending
+  int32_t* plan_pos;        // [cand_nnz][8] score position of (entry, row) in the row's list, or -1
   int rows_bh;              // B * H
   int64_t cand_nnz;
   int N;
@@ -180,43 +185,44 @@ __global__ void __launch_bounds__(kS2Threads, 4) pool_kernel(Stage2Params p) {
 }
 
 // ---------------------------------------------------------------------------
-// Scoring: one CTA per (head, 8 consecutive query blocks).  The union of the 8
-// candidate lists is scored once per key block (each kbar value read feeds 8
-// dot products); every row's scores go to its candidate positions in a global
-// array [BH, cand_nnz] (a row's position of block J = rank of J in the row's
-// sorted list, from per-row bitmaps and prefix popcounts).
+// Scoring, in two kernels.
+//
+// plan_kernel, one CTA per group of 8 consecutive query blocks, from the
+// candidate CSR alone (the same for every head): the union of the 8 candidate
+// lists and, for each (union member J, row r), the position of J in row r's
+// list -- its rank, from per-row bitmaps and prefix popcounts -- or -1 if row
+// r does not list J or needs no score for it.  Union sizes are a fraction of
+// the 8 rows' total, so the entries fit in cand_nnz; a counter hands out the
+// space.
+//
+// score_kernel, one CTA per (head, group): every union member's kbar column is
+// read once and feeds 8 dot products; the scores go to their positions in the
+// per-candidate array [BH, cand_nnz].
 // ---------------------------------------------------------------------------
-__host__ __device__ constexpr size_t score_smem_bytes(int D, int nb) {
-  // qsT [D][8] f32, union bitmap + prefix, 8 row bitmaps + prefixes, 8 "needs a
-  // score" bitmaps, union list
-  return static_cast<size_t>(kSelRows) * D * 4 +
-         static_cast<size_t>((nb + 31) / 32) * 4 * (2 + 3 * kSelRows) + static_cast<size_t>(nb) * 4 + 64;
+__host__ __device__ constexpr size_t plan_smem_bytes(int nb) {
+  // union bitmap + prefix, 8 row bitmaps + prefixes, 8 "needs a score" bitmaps,
+  // union list
+  return static_cast<size_t>((nb + 31) / 32) * 4 * (2 + 3 * kSelRows) + static_cast<size_t>(nb) * 4 + 64;
 }
 
-template <int D>
-__global__ void __launch_bounds__(kS2Threads, 3) score_kernel(Stage2Params p) {
-  extern __shared__ __align__(16) uint8_t sc_smem[];
+__global__ void __launch_bounds__(kS2Threads) plan_kernel(Stage2Params p) {
+  extern __shared__ __align__(16) uint8_t pl_smem[];
   const int nb = p.nb;
   const int nwords = (nb + 31) >> 5;
-  float* qsT = reinterpret_cast<float*>(sc_smem);                       // [D][8]
-  uint32_t* ubits = reinterpret_cast<uint32_t*>(qsT + kSelRows * D);    // [nwords]
-  uint32_t* rbits = ubits + nwords;                                     // [8][nwords]
+  uint32_t* ubits = reinterpret_cast<uint32_t*>(pl_smem);                 // [nwords]
+  uint32_t* rbits = ubits + nwords;                                       // [8][nwords]
   int32_t* upre = reinterpret_cast<int32_t*>(rbits + kSelRows * nwords);  // [nwords]
-  int32_t* rpre = upre + nwords;                                        // [8][nwords]
+  int32_t* rpre = upre + nwords;                                          // [8][nwords]
   uint32_t* nbits = reinterpret_cast<uint32_t*>(rpre + kSelRows * nwords);  // [8][nwords]
   int32_t* ulist = reinterpret_cast<int32_t*>(nbits + kSelRows * nwords);  // [nb]
-  __shared__ int u_total;
+  __shared__ int u_total, u_off;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
-  const int I0 = blockIdx.x * kSelRows;
+  const int grp = blockIdx.x;
+  const int I0 = grp * kSelRows;
   const bool dynamic = p.mode == DYNRAD_DYNAMIC_THRESHOLD;
   // static mode without score export never needs the forced blocks' scores
   const bool skip_forced = !dynamic && p.scores_out == nullptr;
 
-  for (int i = threadIdx.x; i < kSelRows * D; i += kS2Threads) {
-    const int r = i / D, d = i % D;
-    qsT[d * kSelRows + r] = (I0 + r < nb) ? p.qbar[(static_cast<int64_t>(bh) * nb + I0 + r) * D + d] : 0.f;
-  }
   for (int i = threadIdx.x; i < kSelRows * nwords; i += kS2Threads) {
     rbits[i] = 0u;
     nbits[i] = 0u;
@@ -225,10 +231,9 @@ __global__ void __launch_bounds__(kS2Threads, 3) score_kernel(Stage2Params p) {
   // row bitmaps (warp r owns row I0 + r): every candidate (for ranks) and the
   // candidates that need a score
   const int I = I0 + warp;
-  int c_beg = 0, n = 0;
   if (I < nb) {
-    c_beg = p.cand_row_ptr[I];
-    n = p.cand_row_ptr[I + 1] - c_beg;
+    const int c_beg = p.cand_row_ptr[I];
+    const int n = p.cand_row_ptr[I + 1] - c_beg;
     const int flo = p.forced_lo[I], fhi = p.forced_hi[I];
     // the list is sorted, so lanes sharing a bitmap word are adjacent: OR their
     // bits within the warp, one shared-memory update per word
@@ -239,10 +244,10 @@ __global__ void __launch_bounds__(kS2Threads, 3) score_kernel(Stage2Params p) {
       const int w = in ? (J >> 5) : -1 - lane;
       const uint32_t bit = in ? 1u << (J & 31) : 0u;
       const uint32_t need = (in && (!skip_forced || J < flo || J > fhi)) ? bit : 0u;
-      const unsigned grp = __match_any_sync(0xffffffffu, w);
-      const uint32_t all_bits = __reduce_or_sync(grp, bit);
-      const uint32_t need_bits = __reduce_or_sync(grp, need);
-      if (in && lane == __ffs(grp) - 1) {
+      const unsigned grp_lanes = __match_any_sync(0xffffffffu, w);
+      const uint32_t all_bits = __reduce_or_sync(grp_lanes, bit);
+      const uint32_t need_bits = __reduce_or_sync(grp_lanes, need);
+      if (in && lane == __ffs(grp_lanes) - 1) {
         rbits[warp * nwords + w] |= all_bits;
         nbits[warp * nwords + w] |= need_bits;
       }
@@ -278,19 +283,60 @@ __global__ void __launch_bounds__(kS2Threads, 3) score_kernel(Stage2Params p) {
     if (which == kSelRows && lane == 0) u_total = carry;
   }
   __syncthreads();
-  // union list, one word per warp iteration
+  // union list, one word per warp iteration; space for this group's entries
   for (int w = warp; w < nwords; w += kSelRows) {
     const uint32_t bits = ubits[w];
     if ((bits >> lane) & 1u) ulist[upre[w] + __popc(bits & ((1u << lane) - 1u))] = (w << 5) + lane;
   }
+  if (threadIdx.x == 0) {
+    int off = atomicAdd(p.plan_alloc, u_total);
+    if (static_cast<int64_t>(off) + u_total > p.cand_nnz) {   // cannot happen for a valid CSR
+      record_error(DYNRAD_ERR_CAPACITY);
+      off = -1;
+    }
+    u_off = off;
+    p.plan_off[grp] = off < 0 ? 0 : off;
+    p.plan_cnt[grp] = off < 0 ? 0 : u_total;
+  }
   __syncthreads();
-  const int U = u_total;
+  const int U = u_total, off = u_off;
+  if (off < 0) return;
+  for (int u = threadIdx.x; u < U; u += kS2Threads) {
+    const int J = ulist[u];
+    const int w = J >> 5;
+    const uint32_t below = (1u << (J & 31)) - 1u;
+    p.plan_J[off + u] = J;
+    int32_t pos[kSelRows];
+#pragma unroll
+    for (int r = 0; r < kSelRows; ++r) {
+      const bool has = I0 + r < nb && ((nbits[r * nwords + w] >> (J & 31)) & 1u);
+      pos[r] = has ? p.cand_row_ptr[I0 + r] + rpre[r * nwords + w] + __popc(rbits[r * nwords + w] & below) : -1;
+    }
+    int4* dst = reinterpret_cast<int4*>(p.plan_pos + static_cast<int64_t>(off + u) * kSelRows);
+    dst[0] = make_int4(pos[0], pos[1], pos[2], pos[3]);
+    dst[1] = make_int4(pos[4], pos[5], pos[6], pos[7]);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kS2Threads, 3) score_kernel(Stage2Params p) {
+  __shared__ __align__(16) float qsT[D * kSelRows];   // [D][8]
+  const int nb = p.nb;
+  const int bh = blockIdx.y;
+  const int grp = blockIdx.x;
+  const int I0 = grp * kSelRows;
+  for (int i = threadIdx.x; i < kSelRows * D; i += kS2Threads) {
+    const int r = i / D, d = i % D;
+    qsT[d * kSelRows + r] = (I0 + r < nb) ? p.qbar[(static_cast<int64_t>(bh) * nb + I0 + r) * D + d] : 0.f;
+  }
+  __syncthreads();
+  const int U = p.plan_cnt[grp], off = p.plan_off[grp];
   const float* kT = p.kbarT + static_cast<int64_t>(bh) * D * p.nbp;
   float* out = p.scores + static_cast<int64_t>(bh) * p.cand_nnz;
   for (int u0 = threadIdx.x; u0 < U; u0 += 2 * kS2Threads) {
     const int u1 = u0 + kS2Threads;
-    const int J0 = ulist[u0];
-    const int J1 = u1 < U ? ulist[u1] : J0;
+    const int J0 = p.plan_J[off + u0];
+    const int J1 = u1 < U ? p.plan_J[off + u1] : J0;
     float2 a0[4], a1[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
@@ -315,20 +361,19 @@ __global__ void __launch_bounds__(kS2Threads, 3) score_kernel(Stage2Params p) {
       a1[2] = __ffma2_rn(q45, kk1, a1[2]);
       a1[3] = __ffma2_rn(q67, kk1, a1[3]);
     }
-    // scatter to the rows that list each block
+    // scatter to the rows that need each block's score
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       if (e == 1 && u1 >= U) break;
-      const int J = e == 0 ? J0 : J1;
-      const int w = J >> 5;
-      const uint32_t below = (1u << (J & 31)) - 1u;
+      const int u = e == 0 ? u0 : u1;
+      const int4* pp = reinterpret_cast<const int4*>(p.plan_pos + static_cast<int64_t>(off + u) * kSelRows);
+      const int4 pa = __ldg(pp), pb = __ldg(pp + 1);
+      const int pos[kSelRows] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
 #pragma unroll
       for (int r = 0; r < kSelRows; ++r) {
-        const uint32_t bits = rbits[r * nwords + w];
-        if ((nbits[r * nwords + w] >> (J & 31)) & 1u) {
+        if (pos[r] >= 0) {
           const float2 v = e == 0 ? a0[r >> 1] : a1[r >> 1];
-          const float sc = ((r & 1) ? v.y : v.x) * p.scale;
-          out[p.cand_row_ptr[I0 + r] + rpre[r * nwords + w] + __popc(bits & below)] = sc;
+          out[pos[r]] = ((r & 1) ? v.y : v.x) * p.scale;
         }
       }
     }
@@ -342,9 +387,6 @@ __global__ void __launch_bounds__(kS2Threads, 3) score_kernel(Stage2Params p) {
 // ---------------------------------------------------------------------------
 constexpr int kSelWarps = 8;
 
-// DYN: dynamic-threshold mode (fp64 masses as fixed-point weights); otherwise
-// static-ratio mode, where every free block weighs 1 and only the keys are kept
-// in registers.
 template <int E, bool DYN>
 __global__ void __launch_bounds__(kSelWarps * 32, DYN ? (E <= 4 ? 4 : (E <= 8 ? 3 : (E <= 16 ? 2 : 1)))
                                                       : (E <= 8 ? 4 : (E <= 16 ? 3 : 2)))
@@ -522,15 +564,27 @@ __global__ void __launch_bounds__(kSelWarps * 32, DYN ? (E <= 4 ? 4 : (E <= 8 ? 
   uint32_t kept = forced;
   if (!cut_none) {
     uint64_t tie_run = 0;
+    const uint32_t lt_mask = (1u << lane) - 1u;
 #pragma unroll
     for (int i = 0; i < E; ++i) {
       const bool fr = (freev >> i) & 1u;
       bool k_ = fr && (keep_all || key[i] > kstar);
       const bool tie = !keep_all && fr && key[i] == kstar;
-      const uint64_t tw = tie ? wof(i) : 0;
-      const uint64_t ex = warp_excl_scan_u64(tw, lane);
-      if (tie && !reach(above + tie_run + ex)) k_ = true;
-      tie_run += warp_sum_u64(tw);
+      // ties are few (usually the cut element alone): scan only where they are
+      const unsigned tb = __ballot_sync(0xffffffffu, tie);
+      if (tb != 0u) {
+        uint64_t ex, sum;
+        if constexpr (DYN) {
+          const uint64_t tw = tie ? wof(i) : 0;
+          ex = warp_excl_scan_u64(tw, lane);
+          sum = warp_sum_u64(tw);
+        } else {   // unit weights: ranks from the ballot
+          ex = static_cast<uint64_t>(__popc(tb & lt_mask));
+          sum = static_cast<uint64_t>(__popc(tb));
+        }
+        if (tie && !reach(above + tie_run + ex)) k_ = true;
+        tie_run += sum;
+      }
       kept |= (k_ ? 1u : 0u) << i;
     }
   }

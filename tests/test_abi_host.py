@@ -111,8 +111,11 @@ def test_workspace_size_formula():
     rows = 40 * g.n_blocks
     nbp = (g.n_blocks + 31) // 32 * 32
     # qbar [BH, Nb, D] + kbar transposed [BH, D, Nb padded to 32] (fp32) + the
-    # kept lists + scan partials, each 256-byte aligned
-    need = rows * 128 * 4 + 40 * 128 * nbp * 4 + 40 * nnz * 4
+    # kept lists + scan partials + the scoring plan (per group of 8 rows: offset
+    # and size; union members and 8 scatter positions, at most cand_nnz
+    # entries), each 256-byte aligned
+    groups = (g.n_blocks + 7) // 8
+    need = rows * 128 * 4 + 40 * 128 * nbp * 4 + 40 * nnz * 4 + 2 * groups * 4 + 4 + nnz * 4 * 9
     assert need <= ws < need + 4096
 
 
