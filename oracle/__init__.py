@@ -14,7 +14,10 @@ from "DynamicRad: Content-Adaptive Sparse Attention for Long Video Diffusion"
   mean pooling, block proxy scores, static-ratio (top rho, k from Eq. 8) and
   dynamic-threshold (smallest prefix reaching softmax block mass tau);
 * ``attention`` -- Sec. 3.3, Eqs. 12-13 with epsilon -> 0: softmax attention
-  restricted to the kept blocks, with its log-sum-exp.
+  restricted to the kept blocks, with its log-sum-exp;
+* ``sampling``  -- the paper-exact static-ratio mode of Sec. 3.2 (Eq. 8):
+  k = max(1, floor(|P| * rho)) token pairs per frame pair, drawn with a seeded
+  SplitMix64 generator, aggregated to blocks as in Sec. 3.1.
 
 Every function is pinned by ``-m "not gpu"`` tests to closed forms, library
 routines for special cases, brute force on tiny inputs, or invariants the
