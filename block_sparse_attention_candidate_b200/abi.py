@@ -41,6 +41,8 @@ EXPORTED = (
     "dynrad_select_blocks_static_scratch",
     "dynrad_host_path_workspace_bytes",
     "dynrad_host_path",
+    "dynrad_sampled_mask_workspace_bytes",
+    "dynrad_build_sampled_mask",
 )
 
 
@@ -132,6 +134,11 @@ def lib() -> ctypes.CDLL:
         L.dynrad_host_path.restype = ctypes.c_int
         L.dynrad_host_path.argtypes = [_VP, _VP, _VP, _I32, _I32, _I32, _I32, ctypes.POINTER(DynradHostRun), _I32,
                                        _I32, ctypes.c_float, _VP, _SZ, _VP]
+        L.dynrad_sampled_mask_workspace_bytes.restype = _SZ
+        L.dynrad_sampled_mask_workspace_bytes.argtypes = [_GP, _I64]
+        L.dynrad_build_sampled_mask.restype = ctypes.c_int
+        L.dynrad_build_sampled_mask.argtypes = [_GP, ctypes.c_double, ctypes.c_double, ctypes.c_uint64, _VP, _VP, _I64,
+                                                _VP, _VP, _I32, _VP, _VP, _I64, _VP, _VP, _SZ, _VP]
         _lib = L
     return _lib
 
@@ -343,3 +350,28 @@ def dynrad_host_path(q_host, k_host, v_host, runs, chunk_bh=4, scale=0.0, worksp
                                   float(scale), _ptr(ws.view), ws.view.numel(), _stream(stream)),
            "dynrad_host_path")
     return ws
+
+
+def dynrad_build_sampled_mask(geom, cand, rho1, rho2, seed, replicas=1, thresholds=False, stream=None):
+    """Paper-exact static-ratio mask (Eq. 8, seeded token-pair sampling), the
+    same for every head, written ``replicas`` times.  Returns (row_ptr int32
+    [replicas*Nb+1], col_idx int32 with capacity replicas*cand_nnz, thresholds
+    int64 [F*F] holding the uint64 T(i, j) bits, or None)."""
+    L = lib()
+    cg = make_geom(geom)
+    device = cand["row_ptr"].device
+    ws_bytes = int(L.dynrad_sampled_mask_workspace_bytes(ctypes.byref(cg), cand["nnz"]))
+    if ws_bytes == 0:
+        raise DynradError(DYNRAD_ERR_INVALID_ARG, "dynrad_sampled_mask_workspace_bytes")
+    ws = torch.empty(ws_bytes + 256, dtype=torch.uint8, device=device)
+    off = (-ws.data_ptr()) % 256
+    nb = cand["nb"]
+    row_ptr = torch.empty(replicas * nb + 1, dtype=torch.int32, device=device)
+    col = torch.empty(max(1, replicas * cand["nnz"]), dtype=torch.int32, device=device)
+    thr = torch.empty(geom.frames * geom.frames, dtype=torch.int64, device=device) if thresholds else None
+    _check(L.dynrad_build_sampled_mask(ctypes.byref(cg), float(rho1), float(rho2), int(seed) & ((1 << 64) - 1),
+                                       _ptr(cand["row_ptr"]), _ptr(cand["col"]), cand["nnz"], _ptr(cand["forced_lo"]),
+                                       _ptr(cand["forced_hi"]), int(replicas), _ptr(row_ptr), _ptr(col), col.numel(),
+                                       _ptr(thr), ctypes.c_void_p(ws.data_ptr() + off), ws_bytes, _stream(stream)),
+           "dynrad_build_sampled_mask")
+    return row_ptr, col, thr

@@ -15,6 +15,7 @@
 #include "attention.cuh"
 #include "candidates.cuh"
 #include "common.cuh"
+#include "sampling.cuh"
 #include "select.cuh"
 
 using namespace dynrad;
@@ -396,6 +397,119 @@ int dynrad_select_blocks(const void* q, const void* k, int32_t B, int32_t H, int
     compact_kernel<<<static_cast<unsigned>(cblocks), kCompactThreads, 0, st>>>(cp);
     if ((rc = launch_status()) != DYNRAD_OK) return rc;
   }
+  return DYNRAD_OK;
+}
+
+namespace {
+
+struct SampleWorkspace {
+  size_t pairs, hist, thresholds, kept, partial, total;
+};
+
+SampleWorkspace sample_layout(int64_t frames, int64_t nb, int64_t cand_nnz) {
+  SampleWorkspace w;
+  const int64_t fp = frames * frames;
+  const int64_t tiles = (nb + 1 + kScanTile - 1) / kScanTile;
+  w.pairs = 0;
+  w.hist = align256(w.pairs + static_cast<size_t>(fp) * sizeof(SamplePair));
+  w.thresholds = align256(w.hist + static_cast<size_t>(fp) * kSampleBins * 4);
+  w.kept = align256(w.thresholds + static_cast<size_t>(fp) * 8);
+  w.partial = align256(w.kept + static_cast<size_t>(cand_nnz) * 4);
+  w.total = align256(w.partial + static_cast<size_t>(tiles) * 8);
+  return w;
+}
+
+}  // namespace
+
+size_t dynrad_sampled_mask_workspace_bytes(const dynrad_geom* geom, int64_t cand_nnz) {
+  GeomDev g;
+  if (check_geom(geom, &g) != DYNRAD_OK || cand_nnz < 1) return 0;
+  return sample_layout(g.frames, g.nb, cand_nnz).total;
+}
+
+int dynrad_build_sampled_mask(const dynrad_geom* geom, double rho1, double rho2, uint64_t seed,
+                              const int32_t* cand_row_ptr, const int32_t* cand_col, int64_t cand_nnz,
+                              const int32_t* forced_lo, const int32_t* forced_hi, int32_t replicas,
+                              int32_t* row_ptr, int32_t* col_idx, int64_t col_cap, uint64_t* thresholds_out,
+                              void* workspace, size_t workspace_bytes, dynrad_stream_t stream) {
+  GeomDev g;
+  int rc = check_geom(geom, &g);
+  if (rc != DYNRAD_OK) return rc;
+  if (cand_row_ptr == nullptr || cand_col == nullptr || forced_lo == nullptr || forced_hi == nullptr ||
+      row_ptr == nullptr || col_idx == nullptr || workspace == nullptr)
+    return DYNRAD_ERR_INVALID_ARG;
+  if (!(rho1 > 0.0 && rho1 <= 1.0) || !(rho2 > 0.0 && rho2 <= 1.0)) return DYNRAD_ERR_INVALID_ARG;
+  if (cand_nnz < 1 || replicas < 1 || col_cap < 0) return DYNRAD_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DYNRAD_ERR_INVALID_ARG;
+  if (g.block != 32 && g.block != 64 && g.block != 128) return DYNRAD_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(replicas) * g.nb + 1 > INT32_MAX) return DYNRAD_ERR_UNSUPPORTED;
+  if ((static_cast<int64_t>(g.nt) + kSampleRowsPerCta - 1) / kSampleRowsPerCta > 65535) return DYNRAD_ERR_UNSUPPORTED;
+  const SampleWorkspace w = sample_layout(g.frames, g.nb, cand_nnz);
+  if (workspace_bytes < w.total) return DYNRAD_ERR_CAPACITY;
+  cudaStream_t st = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  SampleParams sp;
+  sp.g = g;
+  sp.rho1 = rho1;
+  sp.rho2 = rho2;
+  sp.seed = seed;
+  sp.pairs = reinterpret_cast<SamplePair*>(ws + w.pairs);
+  sp.hist = reinterpret_cast<uint32_t*>(ws + w.hist);
+  sp.thresholds = reinterpret_cast<uint64_t*>(ws + w.thresholds);
+  sp.cand_row_ptr = cand_row_ptr;
+  sp.cand_col = cand_col;
+  sp.forced_lo = forced_lo;
+  sp.forced_hi = forced_hi;
+  sp.counts = row_ptr;
+  sp.kept_tmp = reinterpret_cast<int32_t*>(ws + w.kept);
+  sp.pass = 0;
+  const int fp = g.frames * g.frames;
+  sample_setup_kernel<<<(fp + 255) / 256, 256, 0, st>>>(sp);
+  if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  if (cudaMemsetAsync(sp.hist, 0, static_cast<size_t>(fp) * kSampleBins * 4, st) != cudaSuccess)
+    return DYNRAD_ERR_CUDA;
+  const dim3 hgrid(fp, (g.nt + kSampleRowsPerCta - 1) / kSampleRowsPerCta);
+  for (int pass = 0; pass < kSamplePasses; ++pass) {
+    sp.pass = pass;
+    sample_hist_kernel<<<hgrid, kSampleThreads, 0, st>>>(sp);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+    sample_pick_kernel<<<fp, kSampleThreads, 0, st>>>(sp);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  }
+  const size_t msmem = static_cast<size_t>(g.frames) * 5 + 16;
+  if (g.block == 32) sample_mark_kernel<32><<<g.nb, kSampleThreads, msmem, st>>>(sp);
+  else if (g.block == 64) sample_mark_kernel<64><<<g.nb, kSampleThreads, msmem, st>>>(sp);
+  else sample_mark_kernel<128><<<g.nb, kSampleThreads, msmem, st>>>(sp);
+  if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  // counts -> offsets -> compacted replica 0 -> replicas
+  {
+    const int64_t rows = g.nb;
+    int64_t* partial = reinterpret_cast<int64_t*>(ws + w.partial);
+    const int64_t tiles = (rows + 1 + kScanTile - 1) / kScanTile;
+    scan_partial_kernel<<<static_cast<unsigned>(tiles), kScanThreads, 0, st>>>(row_ptr, rows, partial);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+    CompactParams cp;
+    cp.row_ptr = row_ptr;
+    cp.partial = partial;
+    cp.rows = rows;
+    cp.nb = g.nb;
+    cp.cand_row_ptr = cand_row_ptr;
+    cp.kept_tmp = sp.kept_tmp;
+    cp.cand_nnz = cand_nnz;
+    cp.col_idx = col_idx;
+    cp.col_cap = col_cap;
+    scan_apply_kernel<<<static_cast<unsigned>(tiles), kScanThreads, 0, st>>>(cp);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+    const int64_t cblocks = (rows * 32 + kCompactThreads - 1) / kCompactThreads;
+    compact_kernel<<<static_cast<unsigned>(cblocks), kCompactThreads, 0, st>>>(cp);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+    replicate_csr_kernel<<<264, 256, 0, st>>>(row_ptr, col_idx, g.nb, replicas, col_cap);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  }
+  if (thresholds_out != nullptr &&
+      cudaMemcpyAsync(thresholds_out, sp.thresholds, static_cast<size_t>(fp) * 8, cudaMemcpyDeviceToDevice, st) !=
+          cudaSuccess)
+    return DYNRAD_ERR_CUDA;
   return DYNRAD_OK;
 }
 

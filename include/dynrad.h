@@ -212,6 +212,54 @@ int dynrad_sparse_attn(const void *q, const void *k, const void *v, int32_t B,
                        dynrad_stream_t stream);
 
 /*
+ * Paper-exact static-ratio mode (Sec. 3.2 "Static-ratio mode", Eq. 8): a
+ * content-free, seeded block mask, the same for every (batch, head).
+ *
+ * For each ordered frame pair (i, j) at distance t = |i - j| >= 2 that the
+ * split rule (Eq. 6) keeps, k = max(1, floor(|P(i,j)| * rho)) token pairs of
+ * the candidate set P(i,j) of Eq. 7 are sampled, rho = rho1 when
+ * L(t) >= block (near field) and rho2 when L(t) < block (far field); pairs at
+ * t <= 1 are all kept (rho = 1).  The sample is the k pairs with the smallest
+ * keys, the key of pair (u, v) being output c + 1 of the SplitMix64 generator
+ * seeded with `seed`, c = ((i*F + j)*N_t + u)*N_t + v (keys never tie).  The
+ * sampled token links are aggregated to blocks with (theta_c, theta_m) as for
+ * the candidate set (Sec. 3.1) and united with each row's forced range.  The
+ * mask is a subset of the candidate set; building it costs a few radix passes
+ * over all candidate token pairs (cache it: it depends only on the geometry,
+ * rho1, rho2 and seed).
+ *
+ *   geom, cand_*, forced_*  the geometry and its candidate set / forced ranges
+ *                 from dynrad_build_candidates (DEVICE)
+ *   rho1, rho2    in (0, 1]
+ *   replicas      number of copies of the Nb-row mask written one after the
+ *                 other (B*H, so the result feeds dynrad_sparse_attn directly)
+ *   row_ptr       DEVICE int32 [replicas*Nb + 1]
+ *   col_idx       DEVICE int32, capacity col_cap >= replicas * (kept blocks);
+ *                 replicas * cand_nnz always suffices
+ *   thresholds_out  nullable DEVICE uint64 [F*F]: T(i, j), the largest sampled
+ *                 key of frame pair (i, j) (row-major i*F + j); UINT64_MAX
+ *                 where no sampling happens (t <= 1, pairs the split rule
+ *                 drops)
+ *   workspace     DEVICE, 256-byte aligned, dynrad_sampled_mask_workspace_bytes
+ *                 (geom, cand_nnz) bytes
+ * Errors: DYNRAD_ERR_INVALID_ARG (null pointer, rho out of range, replicas <
+ * 1, misaligned workspace), DYNRAD_ERR_UNSUPPORTED (block not 32/64/128, size
+ * limits), DYNRAD_ERR_CAPACITY (workspace) -- before any launch; a col_idx
+ * capacity exceeded on the device is recorded in the device status.
+ */
+size_t dynrad_sampled_mask_workspace_bytes(const dynrad_geom *geom,
+                                           int64_t cand_nnz);
+int dynrad_build_sampled_mask(const dynrad_geom *geom, double rho1, double rho2,
+                              uint64_t seed, const int32_t *cand_row_ptr,
+                              const int32_t *cand_col, int64_t cand_nnz,
+                              const int32_t *forced_lo,
+                              const int32_t *forced_hi, int32_t replicas,
+                              int32_t *row_ptr, int32_t *col_idx,
+                              int64_t col_cap, uint64_t *thresholds_out,
+                              void *workspace, size_t workspace_bytes,
+                              dynrad_stream_t stream);
+
+/*
  * Stages 2 and 3 from and to HOST memory (no counterpart in the paper: a
  * runtime convenience for callers whose Q, K, V live on the host).
  *

@@ -177,3 +177,46 @@ def aggregate_links(geom, links: np.ndarray):
 def sampled_mask_csr(geom, rho1: float, rho2: float, seed: int):
     """The paper-exact static-ratio block mask (all rows; small geometries)."""
     return aggregate_links(geom, sampled_links(geom, rho1, rho2, seed))
+
+
+def sampled_mask_rows(geom, rho1: float, rho2: float, seed: int, rows, thresholds=None):
+    """Block-mask rows for the given query blocks, by token-level evaluation of
+    the sample restricted to each row's query tokens (large geometries).
+    ``thresholds``: optional dict (i, j) -> T, else computed here.  Returns a
+    list of sorted int64 arrays."""
+    nt = geom.height * geom.width
+    n = geom.frames * nt
+    nb = -(-n // geom.block)
+    l0 = G.base_span(nt)
+    w_t, r_t = G.frame_tables(geom)
+    keys_all = np.arange(n, dtype=np.int64)
+    kj, kv = keys_all // nt, keys_all % nt
+    blk_of_key = keys_all // geom.block
+    n_valid = np.bincount(blk_of_key, minlength=nb)
+    thr = {} if thresholds is None else dict(thresholds)
+    out = []
+    for row in rows:
+        q = np.arange(row * geom.block, min((row + 1) * geom.block, n), dtype=np.int64)
+        col_count = np.zeros(n, dtype=np.int64)
+        near = np.zeros(n, dtype=bool)
+        for qq in q:
+            i, u = divmod(int(qq), nt)
+            t = np.abs(i - kj)
+            in_p = r_t[t] & (np.abs(u - kv) <= w_t[t])
+            sampled = in_p.copy()
+            far = in_p & (t >= 2)
+            for j in np.unique(kj[far]):
+                j = int(j)
+                if (i, j) not in thr:
+                    thr[(i, j)] = frame_pair_threshold(geom, i, j, rho1, rho2, seed)[2]
+                sel = far & (kj == j)
+                ks = pair_keys(seed, geom.frames, nt, i, j, np.full(int(sel.sum()), u), kv[sel])
+                sampled[np.flatnonzero(sel)] = ks <= np.uint64(thr[(i, j)])
+            col_count += sampled
+            near |= (t <= geom.force_t) & r_t[t]
+        active = col_count > geom.theta_c * len(q)
+        n_active = np.bincount(blk_of_key, weights=active, minlength=nb)
+        agg = n_active > geom.theta_m * n_valid
+        forced = np.bincount(blk_of_key, weights=near, minlength=nb) > 0
+        out.append(np.flatnonzero(agg | forced))
+    return out

@@ -189,3 +189,29 @@ def test_host_path_workspace_size_formula():
     # Q, K, V; O and LSE per run; one chunk's kept CSR and selection workspace
     need = 3 * qkv + 4 * (qkv + B * H * N * 4) + (chunk * g.n_blocks + 1) * 4 + chunk * nnz * 4 + sel
     assert need <= got < need + 256 * 16
+
+
+def test_sampled_mask_argument_errors_before_launch():
+    L = abi.lib()
+    geom = WORKLOADS["tiny"].geom
+    g = abi.make_geom(geom)
+    p = ctypes.c_void_p(0x10000)
+    ws = ctypes.c_void_p(0x100000)
+
+    def call(rho1=0.3, rho2=0.1, reps=1, ws_ptr=ws, ws_bytes=1 << 40, rp=p, geom_=g, nnz=100):
+        return L.dynrad_build_sampled_mask(ctypes.byref(geom_), rho1, rho2, 7, p, p, nnz, p, p, reps, rp, p, 1000,
+                                           None, ws_ptr, ws_bytes, None)
+
+    assert call(rp=None) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(rho1=0.0) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(rho2=1.5) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(reps=0) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(nnz=0) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(ws_ptr=ctypes.c_void_p(0x100010)) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(ws_bytes=64) == abi.DYNRAD_ERR_CAPACITY
+    g16 = abi.make_geom(Geometry(4, 4, 4, 16, 0.5, 2.0))
+    assert call(geom_=g16) == abi.DYNRAD_ERR_UNSUPPORTED
+    F = geom.frames
+    need = L.dynrad_sampled_mask_workspace_bytes(ctypes.byref(g), 100)
+    # frame-pair records (48 B), 2048-bin histograms, thresholds, kept lists, scan partials
+    assert F * F * (48 + 2048 * 4 + 8) + 400 <= need < F * F * (48 + 2048 * 4 + 8) + 400 + 256 * 6
