@@ -246,6 +246,11 @@ def main():
     ap.add_argument("--workload", default="wan14b_720p", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sampled", action="store_true",
+                    help="skip the paper-exact static-ratio (seeded sampling) measurement")
+    ap.add_argument("--sampled-rho", default="0.3,0.1", help="rho_1,rho_2 of the sampled static mode")
+    ap.add_argument("--sampled-theta", default="0.2,0.5",
+                    help="theta_c,theta_m (block aggregation) of the sampled static mode")
     ap.add_argument("--e2e-chunk", type=int, default=4,
                     help="(batch, head) rows per chunk of the end-to-end host path")
     ap.add_argument("--no-dense", action="store_true")
@@ -406,6 +411,50 @@ def main():
                  "speedup_vs_dense": {lbl: round(dense_ms / ri["attn_ms"], 2) for lbl, ri in run_info.items()}}
         del rp, col, o, lse
 
+    # ---- paper-exact static-ratio mode (Eq. 8 seeded token-pair sampling): mask
+    # build (content-free, cacheable) and the attention over it
+    sampled = None
+    if not args.no_sampled:
+        rho1, rho2 = (float(x) for x in args.sampled_rho.split(","))
+        th_c, th_m = (float(x) for x in args.sampled_theta.split(","))
+        g0 = replace(runs[0]["geom"], theta_c=th_c, theta_m=th_m)
+        cand0 = abi.dynrad_build_candidates(g0)
+        rp_s, col_s, _ = abi.dynrad_build_sampled_mask(g0, cand0, rho1, rho2, 2026, replicas=B * H)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        reps = 3
+        e0.record(stream)
+        for _ in range(reps):
+            abi.dynrad_build_sampled_mask(g0, cand0, rho1, rho2, 2026, replicas=B * H)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        build_ms = e0.elapsed_time(e1) / reps
+        o_s = torch.empty_like(q)
+        lse_s = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        for _ in range(2):
+            abi.dynrad_sparse_attn(q, k, v, g0.block, rp_s, col_s, out=o_s, lse=lse_s)
+        e0.record(stream)
+        for _ in range(reps):
+            abi.dynrad_sparse_attn(q, k, v, g0.block, rp_s, col_s, out=o_s, lse=lse_s)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        st = abi.dynrad_device_status(clear=True)
+        if st != 0:
+            raise RuntimeError(f"device status after the sampled-mask run: {abi.status_string(st)}")
+        attn_s = e0.elapsed_time(e1) / reps
+        rpn = rp_s.cpu().numpy().astype(np.int64)
+        coln = col_s[: int(rpn[-1])].cpu().numpy().astype(np.int64)
+        fl = kept_flops(rpn, coln, N, g0.block, B * H, D)
+        nb0 = g0.n_blocks
+        sampled = {"rho1": rho1, "rho2": rho2, "theta_c": th_c, "theta_m": th_m, "seed": 2026, "gamma": g0.gamma,
+                   "mask_build_ms": round(build_ms, 3), "attn_ms": round(attn_s, 3),
+                   "attn_tflops": round(fl / (attn_s * 1e-3) / 1e12, 1),
+                   "block_density": round(int(rpn[-1]) / (B * H * nb0 * nb0), 4),
+                   "candidate_density": round(cand0["nnz"] / (nb0 * nb0), 4),
+                   "speedup_vs_dense": round(dense["ms"] / attn_s, 2) if dense else None}
+        del rp_s, col_s, o_s, lse_s
+
     # ---- end to end through the host-memory entry point: pinned host Q, K, V
     # in, every run's O and LSE back to pinned host memory, the copies
     # overlapped with the kernels by dynrad_host_path (chunks of heads)
@@ -474,6 +523,7 @@ def main():
         "clocks": clocks,
         "runs": run_info,
         "dense_same_kernel": dense,
+        "sampled_static": sampled,
         "stage_ms_per_step": {"candidates": round(float(stage_ms[:, 0].sum()), 4),
                               "selection": round(float(stage_ms[:, 1].sum()), 4),
                               "attention": round(attn_ms_total, 4)},
