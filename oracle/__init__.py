@@ -17,7 +17,11 @@ from "DynamicRad: Content-Adaptive Sparse Attention for Long Video Diffusion"
   restricted to the kept blocks, with its log-sum-exp;
 * ``sampling``  -- the paper-exact static-ratio mode of Sec. 3.2 (Eq. 8):
   k = max(1, floor(|P| * rho)) token pairs per frame pair, drawn with a seeded
-  SplitMix64 generator, aggregated to blocks as in Sec. 3.1.
+  SplitMix64 generator, aggregated to blocks as in Sec. 3.1;
+* ``dynamic_tokens`` -- the paper-exact dynamic-threshold mode of Sec. 3.2
+  (Eqs. 9-11, Eq. 19): fused-head proxy logits on the candidate token pairs,
+  per-frame-pair z-scores, tau_1 / tau_2 thresholds with the top-pair
+  fallback, aggregated to blocks.
 
 Every function is pinned by ``-m "not gpu"`` tests to closed forms, library
 routines for special cases, brute force on tiny inputs, or invariants the
