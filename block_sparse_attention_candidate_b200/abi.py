@@ -43,6 +43,8 @@ EXPORTED = (
     "dynrad_host_path",
     "dynrad_sampled_mask_workspace_bytes",
     "dynrad_build_sampled_mask",
+    "dynrad_token_mask_workspace_bytes",
+    "dynrad_build_token_mask",
 )
 
 
@@ -139,6 +141,12 @@ def lib() -> ctypes.CDLL:
         L.dynrad_build_sampled_mask.restype = ctypes.c_int
         L.dynrad_build_sampled_mask.argtypes = [_GP, ctypes.c_double, ctypes.c_double, ctypes.c_uint64, _VP, _VP, _I64,
                                                 _VP, _VP, _I32, _VP, _VP, _I64, _VP, _VP, _SZ, _VP]
+        L.dynrad_token_mask_workspace_bytes.restype = _SZ
+        L.dynrad_token_mask_workspace_bytes.argtypes = [_I32, _I32, _GP, _I64]
+        L.dynrad_build_token_mask.restype = ctypes.c_int
+        L.dynrad_build_token_mask.argtypes = [_VP, _VP, _I32, _I32, _I32, _I32, _I32, _GP, ctypes.c_double,
+                                              ctypes.c_double, _VP, _VP, _I64, _VP, _VP, _VP, _VP, _I64, _VP, _VP,
+                                              _SZ, _VP]
         _lib = L
     return _lib
 
@@ -375,3 +383,31 @@ def dynrad_build_sampled_mask(geom, cand, rho1, rho2, seed, replicas=1, threshol
                                        _ptr(thr), ctypes.c_void_p(ws.data_ptr() + off), ws_bytes, _stream(stream)),
            "dynrad_build_sampled_mask")
     return row_ptr, col, thr
+
+
+def dynrad_build_token_mask(q, k, geom, cand, tau1, tau2, hf=2, stats=False, stream=None):
+    """Paper-exact dynamic-threshold mask (Eqs. 9-11, 19) from bf16 [B, H, N, D]
+    CUDA q, k: one mask per batch element from its first ``hf`` heads, written
+    for every head.  Returns (row_ptr int32 [B*H*Nb+1], col_idx int32 with
+    capacity B*H*cand_nnz, stats float64 [B, F*F, 3] (mu, sigma, threshold) or None)."""
+    _require_cuda(q, k)
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16:
+        raise ValueError("q, k must be bf16")
+    B, H, N, D = q.shape
+    L = lib()
+    cg = make_geom(geom)
+    ws_bytes = int(L.dynrad_token_mask_workspace_bytes(B, N, ctypes.byref(cg), cand["nnz"]))
+    if ws_bytes == 0:
+        raise DynradError(DYNRAD_ERR_INVALID_ARG, "dynrad_token_mask_workspace_bytes")
+    ws = torch.empty(ws_bytes + 256, dtype=torch.uint8, device=q.device)
+    off = (-ws.data_ptr()) % 256
+    nb = cand["nb"]
+    row_ptr = torch.empty(B * H * nb + 1, dtype=torch.int32, device=q.device)
+    col = torch.empty(max(1, B * H * cand["nnz"]), dtype=torch.int32, device=q.device)
+    st = torch.empty((B, geom.frames * geom.frames, 3), dtype=torch.float64, device=q.device) if stats else None
+    _check(L.dynrad_build_token_mask(_ptr(q), _ptr(k), B, H, N, D, int(hf), ctypes.byref(cg), float(tau1), float(tau2),
+                                     _ptr(cand["row_ptr"]), _ptr(cand["col"]), cand["nnz"], _ptr(cand["forced_lo"]),
+                                     _ptr(cand["forced_hi"]), _ptr(row_ptr), _ptr(col), col.numel(), _ptr(st),
+                                     ctypes.c_void_p(ws.data_ptr() + off), ws_bytes, _stream(stream)),
+           "dynrad_build_token_mask")
+    return row_ptr, col, st

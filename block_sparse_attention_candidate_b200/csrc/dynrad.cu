@@ -15,6 +15,7 @@
 #include "attention.cuh"
 #include "candidates.cuh"
 #include "common.cuh"
+#include "dyntok.cuh"
 #include "sampling.cuh"
 #include "select.cuh"
 
@@ -510,6 +511,142 @@ int dynrad_build_sampled_mask(const dynrad_geom* geom, double rho1, double rho2,
       cudaMemcpyAsync(thresholds_out, sp.thresholds, static_cast<size_t>(fp) * 8, cudaMemcpyDeviceToDevice, st) !=
           cudaSuccess)
     return DYNRAD_ERR_CUDA;
+  return DYNRAD_OK;
+}
+
+namespace {
+
+struct TokWorkspace {
+  size_t stats, best, thr, colcnt, zero_end, kept, src_ptr, src_col, partial, total;
+};
+
+TokWorkspace tok_layout(int64_t B, int64_t frames, int64_t nb, int64_t n, int64_t cand_nnz) {
+  TokWorkspace w;
+  const int64_t fp = B * frames * frames;
+  const int64_t rows = B * nb;
+  const int64_t tiles = (rows + 1 + kScanTile - 1) / kScanTile;
+  w.stats = 0;
+  w.best = align256(w.stats + static_cast<size_t>(fp) * 16);
+  w.thr = align256(w.best + static_cast<size_t>(fp) * 8);
+  w.colcnt = align256(w.thr + static_cast<size_t>(fp) * 8);
+  w.zero_end = w.colcnt + static_cast<size_t>(rows) * n * 4;
+  w.kept = align256(w.zero_end);
+  w.src_ptr = align256(w.kept + static_cast<size_t>(B * cand_nnz) * 4);
+  w.src_col = align256(w.src_ptr + static_cast<size_t>(rows + 1) * 4);
+  w.partial = align256(w.src_col + static_cast<size_t>(B * cand_nnz) * 4);
+  w.total = align256(w.partial + static_cast<size_t>(tiles) * 8);
+  return w;
+}
+
+constexpr int kTokMaxFusedHeads = 4;
+
+}  // namespace
+
+size_t dynrad_token_mask_workspace_bytes(int32_t B, int32_t N, const dynrad_geom* geom, int64_t cand_nnz) {
+  GeomDev g;
+  if (check_geom(geom, &g) != DYNRAD_OK || B < 1 || N != g.n || cand_nnz < 1) return 0;
+  return tok_layout(B, g.frames, g.nb, g.n, cand_nnz).total;
+}
+
+int dynrad_build_token_mask(const void* q, const void* k, int32_t B, int32_t H, int32_t N, int32_t D, int32_t hf,
+                            const dynrad_geom* geom, double tau1, double tau2, const int32_t* cand_row_ptr,
+                            const int32_t* cand_col, int64_t cand_nnz, const int32_t* forced_lo,
+                            const int32_t* forced_hi, int32_t* row_ptr, int32_t* col_idx, int64_t col_cap,
+                            double* stats_out, void* workspace, size_t workspace_bytes, dynrad_stream_t stream) {
+  GeomDev g;
+  int rc = check_geom(geom, &g);
+  if (rc != DYNRAD_OK) return rc;
+  if (q == nullptr || k == nullptr || cand_row_ptr == nullptr || cand_col == nullptr || forced_lo == nullptr ||
+      forced_hi == nullptr || row_ptr == nullptr || col_idx == nullptr || workspace == nullptr)
+    return DYNRAD_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N != g.n || cand_nnz < 1 || col_cap < 0) return DYNRAD_ERR_INVALID_ARG;
+  if (hf < 1 || hf > H || !std::isfinite(tau1) || !std::isfinite(tau2)) return DYNRAD_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DYNRAD_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return DYNRAD_ERR_UNSUPPORTED;
+  if (hf > kTokMaxFusedHeads) return DYNRAD_ERR_UNSUPPORTED;
+  if (g.block != 32 && g.block != 64 && g.block != 128) return DYNRAD_ERR_UNSUPPORTED;
+  if (g.nt > 65535 || B > 65535) return DYNRAD_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * H * g.nb + 1 > INT32_MAX || static_cast<int64_t>(B) * cand_nnz > INT32_MAX)
+    return DYNRAD_ERR_UNSUPPORTED;
+  const TokWorkspace w = tok_layout(B, g.frames, g.nb, g.n, cand_nnz);
+  if (workspace_bytes < w.total) return DYNRAD_ERR_CAPACITY;
+  cudaStream_t st = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DynTokParams tp;
+  tp.g = g;
+  tp.q = static_cast<const __nv_bfloat16*>(q);
+  tp.k = static_cast<const __nv_bfloat16*>(k);
+  tp.B = B;
+  tp.H = H;
+  tp.D = D;
+  tp.hf = hf;
+  tp.tau1 = tau1;
+  tp.tau2 = tau2;
+  tp.inv = 1.0f / (static_cast<float>(hf) * std::sqrt(static_cast<float>(D)));
+  tp.stats = reinterpret_cast<double*>(ws + w.stats);
+  tp.best = reinterpret_cast<unsigned long long*>(ws + w.best);
+  tp.thr = reinterpret_cast<double*>(ws + w.thr);
+  tp.colcnt = reinterpret_cast<uint32_t*>(ws + w.colcnt);
+  tp.cand_row_ptr = cand_row_ptr;
+  tp.cand_col = cand_col;
+  tp.forced_lo = forced_lo;
+  tp.forced_hi = forced_hi;
+  int32_t* src_ptr = reinterpret_cast<int32_t*>(ws + w.src_ptr);
+  int32_t* src_col = reinterpret_cast<int32_t*>(ws + w.src_col);
+  tp.counts = src_ptr;
+  tp.kept_tmp = reinterpret_cast<int32_t*>(ws + w.kept);
+  tp.cand_nnz = cand_nnz;
+  if (cudaMemsetAsync(ws, 0, w.zero_end, st) != cudaSuccess) return DYNRAD_ERR_CUDA;
+  const size_t tsmem = static_cast<size_t>(hf) * D * (kTokRows + kTokCols) * 4;
+  const void* tk = D == 128 ? reinterpret_cast<const void*>(dyntok_tile_kernel<128>)
+                            : reinterpret_cast<const void*>(dyntok_tile_kernel<64>);
+  if (cudaFuncSetAttribute(tk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(tsmem)) != cudaSuccess)
+    return DYNRAD_ERR_CUDA;
+  const int fp = g.frames * g.frames;
+  const dim3 tgrid(fp, (g.nt + kTokRows - 1) / kTokRows, B);
+  for (int pass = 0; pass < 2; ++pass) {
+    tp.pass = pass;
+    if (D == 128)
+      dyntok_tile_kernel<128><<<tgrid, kTokThreads, tsmem, st>>>(tp);
+    else
+      dyntok_tile_kernel<64><<<tgrid, kTokThreads, tsmem, st>>>(tp);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+    if (pass == 0) {
+      const int64_t m = static_cast<int64_t>(B) * fp;
+      dyntok_finalize_kernel<<<static_cast<unsigned>((m + 255) / 256), 256, 0, st>>>(tp, stats_out);
+      if ((rc = launch_status()) != DYNRAD_OK) return rc;
+    }
+  }
+  const size_t asmem = static_cast<size_t>(g.frames) * 5 + 16;
+  const dim3 agrid(g.nb, B);
+  if (g.block == 32) dyntok_aggregate_kernel<32><<<agrid, kTokThreads, asmem, st>>>(tp);
+  else if (g.block == 64) dyntok_aggregate_kernel<64><<<agrid, kTokThreads, asmem, st>>>(tp);
+  else dyntok_aggregate_kernel<128><<<agrid, kTokThreads, asmem, st>>>(tp);
+  if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  {
+    const int64_t rows = static_cast<int64_t>(B) * g.nb;
+    int64_t* partial = reinterpret_cast<int64_t*>(ws + w.partial);
+    const int64_t tiles = (rows + 1 + kScanTile - 1) / kScanTile;
+    scan_partial_kernel<<<static_cast<unsigned>(tiles), kScanThreads, 0, st>>>(src_ptr, rows, partial);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+    CompactParams cp;
+    cp.row_ptr = src_ptr;
+    cp.partial = partial;
+    cp.rows = rows;
+    cp.nb = g.nb;
+    cp.cand_row_ptr = cand_row_ptr;
+    cp.kept_tmp = tp.kept_tmp;
+    cp.cand_nnz = cand_nnz;
+    cp.col_idx = src_col;
+    cp.col_cap = static_cast<int64_t>(B) * cand_nnz;
+    scan_apply_kernel<<<static_cast<unsigned>(tiles), kScanThreads, 0, st>>>(cp);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+    const int64_t cblocks = (rows * 32 + kCompactThreads - 1) / kCompactThreads;
+    compact_kernel<<<static_cast<unsigned>(cblocks), kCompactThreads, 0, st>>>(cp);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+    expand_csr_kernel<<<264, 256, 0, st>>>(src_ptr, src_col, B, H, g.nb, row_ptr, col_idx, col_cap);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  }
   return DYNRAD_OK;
 }
 

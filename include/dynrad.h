@@ -260,6 +260,50 @@ int dynrad_build_sampled_mask(const dynrad_geom *geom, double rho1, double rho2,
                               dynrad_stream_t stream);
 
 /*
+ * Paper-exact dynamic-threshold mode (Sec. 3.2 "Dynamic-threshold mode",
+ * Eqs. 9-11; the fused-head proxy of Eq. 19): a block mask per batch element,
+ * shared by its heads, from token-level proxy logits.
+ *
+ * For every candidate token pair (u, v) of an ordered frame pair (i, j) at
+ * t >= 2 kept by the split rule: s = (1/hf) sum_{h < hf} q_u^h . k_v^h /
+ * sqrt(D) over the FIRST hf heads (fp32 FMAs, fixed order); per frame pair,
+ * mu and the population sigma of s over P(i, j) (fp64 sums); the pair is kept
+ * when (s - mu) / (sigma + 1e-6) > tau, tau = tau1 when L(t) >= block, tau2
+ * otherwise; if none passes, the pair with the largest s (smallest u*N_t + v
+ * among equals) is kept.  Pairs at t <= 1 are all kept.  Kept links are
+ * aggregated with (theta_c, theta_m) and united with the forced range.
+ *
+ *   q, k          DEVICE bf16 [B, H, N, D]; D = 64 or 128; hf in [1, min(H, 4)]
+ *   tau1, tau2    finite z-score thresholds (near / far field)
+ *   cand_*, forced_*  from dynrad_build_candidates for geom (DEVICE)
+ *   row_ptr       DEVICE int32 [B*H*Nb + 1], rows (b, h, I); every head of a
+ *                 batch element gets that element's mask
+ *   col_idx       DEVICE int32, capacity col_cap (B*H*cand_nnz always suffices)
+ *   stats_out     nullable DEVICE double [B][F*F][3]: mu, sigma and the score
+ *                 threshold mu + tau (sigma + 1e-6) per (batch, frame pair);
+ *                 zeros / -inf where nothing is thresholded (t <= 1, dropped)
+ *   workspace     DEVICE, 256-byte aligned, dynrad_token_mask_workspace_bytes
+ *                 (B, N, geom, cand_nnz) bytes (holds a B x Nb x N counter
+ *                 array: ~360 MB per batch element at 75,600 tokens, block 64)
+ * Errors: DYNRAD_ERR_INVALID_ARG / UNSUPPORTED / CAPACITY before any launch
+ * (null pointer, hf out of range, non-finite tau, D, block, N_t > 65535);
+ * a col_idx capacity exceeded on the device is recorded in the device status.
+ */
+size_t dynrad_token_mask_workspace_bytes(int32_t B, int32_t N,
+                                         const dynrad_geom *geom,
+                                         int64_t cand_nnz);
+int dynrad_build_token_mask(const void *q, const void *k, int32_t B, int32_t H,
+                            int32_t N, int32_t D, int32_t hf,
+                            const dynrad_geom *geom, double tau1, double tau2,
+                            const int32_t *cand_row_ptr,
+                            const int32_t *cand_col, int64_t cand_nnz,
+                            const int32_t *forced_lo, const int32_t *forced_hi,
+                            int32_t *row_ptr, int32_t *col_idx,
+                            int64_t col_cap, double *stats_out,
+                            void *workspace, size_t workspace_bytes,
+                            dynrad_stream_t stream);
+
+/*
  * Stages 2 and 3 from and to HOST memory (no counterpart in the paper: a
  * runtime convenience for callers whose Q, K, V live on the host).
  *

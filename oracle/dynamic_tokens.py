@@ -106,3 +106,72 @@ def dynamic_links(geom, qf, kf, tau1: float, tau2: float):
 def dynamic_mask_csr(geom, qf, kf, tau1: float, tau2: float):
     """The paper-exact dynamic-threshold block mask of one batch element."""
     return aggregate_links(geom, dynamic_links(geom, qf, kf, tau1, tau2))
+
+
+def frame_pair_logits(qf, kf, i: int, j: int, nt: int):
+    """Dense [N_t, N_t] proxy logits of frame pair (i, j) (Eq. 9), float64."""
+    hf, _, d = qf.shape
+    acc = np.zeros((nt, nt))
+    for h in range(hf):
+        acc += qf[h, i * nt:(i + 1) * nt] @ kf[h, j * nt:(j + 1) * nt].T
+    return acc / hf / math.sqrt(d)
+
+
+def dynamic_mask_rows(geom, qf, kf, tau1: float, tau2: float, rows, tau_shift: float = 0.0):
+    """Mask rows for the given query blocks (large geometries): per frame pair the
+    logits over P from a dense product, the z-rule at tau + tau_shift, the
+    fallback, then the aggregation restricted to each row's query tokens."""
+    nt = geom.height * geom.width
+    n = geom.frames * nt
+    nb = -(-n // geom.block)
+    w_t, r_t = G.frame_tables(geom)
+    blk_of_key = np.arange(n, dtype=np.int64) // geom.block
+    n_valid = np.bincount(blk_of_key, minlength=nb)
+    uu = np.arange(nt)
+    cache = {}
+
+    def kept_matrix(i, j):
+        if (i, j) in cache:
+            return cache[(i, j)]
+        t = abs(i - j)
+        if not r_t[t]:
+            m = np.zeros((nt, nt), dtype=bool)
+        else:
+            w = w_t[t]
+            inb = np.abs(uu[:, None] - uu[None, :]) <= w
+            tau = threshold(geom, t, tau1, tau2)
+            if tau == -math.inf:
+                m = inb
+            else:
+                s = frame_pair_logits(qf, kf, i, j, nt)
+                sv = s[inb]
+                mu = float(sv.mean())
+                sigma = float(np.sqrt(((sv - mu) ** 2).mean()))
+                m = inb & ((s - mu) / (sigma + EPS_Z) > tau + tau_shift)
+                if not m.any():
+                    flat = np.where(inb, s, -np.inf)
+                    best = int(np.argmax(flat))          # first maximum in (u, v) order
+                    m = np.zeros((nt, nt), dtype=bool)
+                    m.flat[best] = True
+        cache[(i, j)] = m
+        return m
+
+    out = []
+    for row in rows:
+        q = np.arange(row * geom.block, min((row + 1) * geom.block, n), dtype=np.int64)
+        col_count = np.zeros(n, dtype=np.int64)
+        near = np.zeros(n, dtype=bool)
+        for qq in q:
+            i, u = divmod(int(qq), nt)
+            for j in range(geom.frames):
+                m = kept_matrix(i, j)
+                col_count[j * nt:(j + 1) * nt] += m[u]
+                t = abs(i - j)
+                if t <= geom.force_t and r_t[t]:
+                    near[j * nt:(j + 1) * nt] = True
+        active = col_count > geom.theta_c * len(q)
+        n_active = np.bincount(blk_of_key, weights=active, minlength=nb)
+        agg = n_active > geom.theta_m * n_valid
+        forced = np.bincount(blk_of_key, weights=near, minlength=nb) > 0
+        out.append(np.flatnonzero(agg | forced))
+    return out

@@ -215,3 +215,33 @@ def test_sampled_mask_argument_errors_before_launch():
     need = L.dynrad_sampled_mask_workspace_bytes(ctypes.byref(g), 100)
     # frame-pair records (48 B), 2048-bin histograms, thresholds, kept lists, scan partials
     assert F * F * (48 + 2048 * 4 + 8) + 400 <= need < F * F * (48 + 2048 * 4 + 8) + 400 + 256 * 6
+
+
+def test_token_mask_argument_errors_before_launch():
+    L = abi.lib()
+    geom = WORKLOADS["tiny"].geom
+    g = abi.make_geom(geom)
+    p = ctypes.c_void_p(0x10000)
+    ws = ctypes.c_void_p(0x100000)
+    n = geom.n_tokens
+
+    def call(q=p, B=1, H=2, N=n, D=64, hf=2, tau1=0.5, tau2=1.0, ws_ptr=ws, ws_bytes=1 << 40, geom_=g):
+        return L.dynrad_build_token_mask(q, p, B, H, N, D, hf, ctypes.byref(geom_), tau1, tau2, p, p, 100, p, p,
+                                         p, p, 1000, None, ws_ptr, ws_bytes, None)
+
+    assert call(q=None) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(N=n + 1) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(hf=0) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(hf=3) == abi.DYNRAD_ERR_INVALID_ARG            # more fused heads than heads
+    assert call(H=8, hf=5) == abi.DYNRAD_ERR_UNSUPPORTED
+    assert call(tau1=float("inf")) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(D=96) == abi.DYNRAD_ERR_UNSUPPORTED
+    assert call(ws_ptr=ctypes.c_void_p(0x100008)) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(ws_bytes=1024) == abi.DYNRAD_ERR_CAPACITY
+    assert call(geom_=abi.make_geom(Geometry(4, 4, 4, 16, 0.5, 2.0)), N=64) == abi.DYNRAD_ERR_UNSUPPORTED
+    need = L.dynrad_token_mask_workspace_bytes(2, n, ctypes.byref(g), 100)
+    F, nb = geom.frames, geom.n_blocks
+    # per (batch, frame pair) sums, maxima and thresholds; per (batch, row, key
+    # token) link counters; kept lists, per-batch CSR, scan partials
+    base = 2 * F * F * 32 + 2 * nb * n * 4 + 2 * 100 * 4 * 2 + (2 * nb + 1) * 4 + 8
+    assert base <= need < base + 256 * 9
