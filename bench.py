@@ -251,6 +251,11 @@ def main():
     ap.add_argument("--sampled-rho", default="0.3,0.1", help="rho_1,rho_2 of the sampled static mode")
     ap.add_argument("--sampled-theta", default="0.2,0.5",
                     help="theta_c,theta_m (block aggregation) of the sampled static mode")
+    ap.add_argument("--no-token", action="store_true",
+                    help="skip the paper-exact dynamic-threshold (token-level) measurement")
+    ap.add_argument("--token-tau", default="0.0,1.0", help="tau_1,tau_2 of the token-level dynamic mode")
+    ap.add_argument("--token-theta", default="0.2,0.5",
+                    help="theta_c,theta_m (block aggregation) of the token-level dynamic mode")
     ap.add_argument("--e2e-chunk", type=int, default=4,
                     help="(batch, head) rows per chunk of the end-to-end host path")
     ap.add_argument("--no-dense", action="store_true")
@@ -455,6 +460,50 @@ def main():
                    "speedup_vs_dense": round(dense["ms"] / attn_s, 2) if dense else None}
         del rp_s, col_s, o_s, lse_s
 
+    # ---- paper-exact dynamic-threshold mode (Eqs. 9-11, 19: token-level proxy
+    # logits of the first two heads): mask build and the attention over it
+    token = None
+    if not args.no_token:
+        t1, t2 = (float(x) for x in args.token_tau.split(","))
+        th_c, th_m = (float(x) for x in args.token_theta.split(","))
+        g0 = replace(runs[0]["geom"], theta_c=th_c, theta_m=th_m)
+        cand0 = abi.dynrad_build_candidates(g0)
+        rp_t, col_t, _ = abi.dynrad_build_token_mask(q, k, g0, cand0, t1, t2, hf=2)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        reps = 3
+        e0.record(stream)
+        for _ in range(reps):
+            abi.dynrad_build_token_mask(q, k, g0, cand0, t1, t2, hf=2)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        build_ms = e0.elapsed_time(e1) / reps
+        o_t = torch.empty_like(q)
+        lse_t = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        for _ in range(2):
+            abi.dynrad_sparse_attn(q, k, v, g0.block, rp_t, col_t, out=o_t, lse=lse_t)
+        e0.record(stream)
+        for _ in range(reps):
+            abi.dynrad_sparse_attn(q, k, v, g0.block, rp_t, col_t, out=o_t, lse=lse_t)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        st = abi.dynrad_device_status(clear=True)
+        if st != 0:
+            raise RuntimeError(f"device status after the token-mask run: {abi.status_string(st)}")
+        attn_t = e0.elapsed_time(e1) / reps
+        rpn = rp_t.cpu().numpy().astype(np.int64)
+        coln = col_t[: int(rpn[-1])].cpu().numpy().astype(np.int64)
+        fl = kept_flops(rpn, coln, N, g0.block, B * H, D)
+        nb0 = g0.n_blocks
+        token = {"tau1": t1, "tau2": t2, "theta_c": th_c, "theta_m": th_m, "fused_heads": 2, "gamma": g0.gamma,
+                 "mask_build_ms": round(build_ms, 3), "attn_ms": round(attn_t, 3),
+                 "attn_tflops": round(fl / (attn_t * 1e-3) / 1e12, 1),
+                 "block_density": round(int(rpn[-1]) / (B * H * nb0 * nb0), 4),
+                 "candidate_density": round(cand0["nnz"] / (nb0 * nb0), 4),
+                 "speedup_vs_dense": round(dense["ms"] / attn_t, 2) if dense else None}
+        del rp_t, col_t, o_t, lse_t
+
     # ---- end to end through the host-memory entry point: pinned host Q, K, V
     # in, every run's O and LSE back to pinned host memory, the copies
     # overlapped with the kernels by dynrad_host_path (chunks of heads)
@@ -524,6 +573,7 @@ def main():
         "runs": run_info,
         "dense_same_kernel": dense,
         "sampled_static": sampled,
+        "token_dynamic": token,
         "stage_ms_per_step": {"candidates": round(float(stage_ms[:, 0].sum()), 4),
                               "selection": round(float(stage_ms[:, 1].sum()), 4),
                               "attention": round(attn_ms_total, 4)},
