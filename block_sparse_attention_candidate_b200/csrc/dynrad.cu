@@ -561,6 +561,7 @@ int dynrad_build_token_mask(const void* q, const void* k, int32_t B, int32_t H, 
     return DYNRAD_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N != g.n || cand_nnz < 1 || col_cap < 0) return DYNRAD_ERR_INVALID_ARG;
   if (hf < 1 || hf > H || !std::isfinite(tau1) || !std::isfinite(tau2)) return DYNRAD_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k)) return DYNRAD_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DYNRAD_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return DYNRAD_ERR_UNSUPPORTED;
   if (hf > kTokMaxFusedHeads) return DYNRAD_ERR_UNSUPPORTED;
@@ -597,7 +598,7 @@ int dynrad_build_token_mask(const void* q, const void* k, int32_t B, int32_t H, 
   tp.kept_tmp = reinterpret_cast<int32_t*>(ws + w.kept);
   tp.cand_nnz = cand_nnz;
   if (cudaMemsetAsync(ws, 0, w.zero_end, st) != cudaSuccess) return DYNRAD_ERR_CUDA;
-  const size_t tsmem = static_cast<size_t>(hf) * D * (kTokRows + kTokCols) * 4;
+  const size_t tsmem = static_cast<size_t>(tok_row_stride(hf * D)) * (kTokRows + kTokCols) * 2;
   const void* tk = D == 128 ? reinterpret_cast<const void*>(dyntok_tile_kernel<128>)
                             : reinterpret_cast<const void*>(dyntok_tile_kernel<64>);
   if (cudaFuncSetAttribute(tk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(tsmem)) != cudaSuccess)

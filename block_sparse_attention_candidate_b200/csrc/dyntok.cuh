@@ -14,8 +14,8 @@
 //
 // Kernels:
 //   dyntok_tile_kernel<D>   one CTA per (frame pair, 32 rows u, batch): the
-//       32 x 64 logit tiles of the band |u - v| <= w, fp32 FMAs in a fixed
-//       order (identical in both passes).  Pass 0 accumulates sum, sum of
+//       32 x 64 logit tiles of the band |u - v| <= w, bf16 tensor-core MMAs
+//       with fp32 accumulation in a fixed order (identical in both passes).  Pass 0 accumulates sum, sum of
 //       squares (fp64) and the packed maximum; pass 1 counts kept links per
 //       (query block, key token).
 //   dyntok_finalize_kernel  per (batch, frame pair): mu, sigma, the score
@@ -68,9 +68,34 @@ __device__ __forceinline__ float tok_key_to_float(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
+// Row stride (bf16 elements) of the staged Q / K rows: 8 elements of padding
+// keep the 8 rows an ldmatrix reads in distinct bank groups.
+__host__ __device__ constexpr int tok_row_stride(int x) { return x + 8; }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D += A(16x16, row) B(16x8, col), bf16 inputs, fp32 accumulation.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The logit tiles are dense 32 x 64 x (H_f * D) products: warp-level bf16
+// tensor-core MMAs (m16n8k16, fp32 accumulation) on Q / K rows staged in shared
+// memory.  The kernel is bound by moving the band's K rows through L2, so the
+// warp-level instruction suffices.  Warp w computes rows 16 (w / 4) .. +15 and
+// columns 16 (w % 4) .. +15 of the tile, in one fixed k order in both passes.
 template <int D>
 __global__ void __launch_bounds__(kTokThreads) dyntok_tile_kernel(DynTokParams p) {
-  extern __shared__ __align__(16) float tok_smem[];
+  extern __shared__ __align__(16) __nv_bfloat16 tok_smem[];
   const GeomDev& g = p.g;
   const int F = g.frames, nt = g.nt;
   const int pi = blockIdx.x, b = blockIdx.z;
@@ -81,61 +106,65 @@ __global__ void __launch_bounds__(kTokThreads) dyntok_tile_kernel(DynTokParams p
   const int u0 = blockIdx.y * kTokRows;
   if (u0 >= nt) return;
   const int X = p.hf * D;                          // dot-product length
-  float* qT = tok_smem;                            // [X][kTokRows]
-  float* kT = qT + X * kTokRows;                   // [X][kTokCols]
+  const int RS = tok_row_stride(X);
+  __nv_bfloat16* qs = tok_smem;                    // [kTokRows][RS]
+  __nv_bfloat16* ks = qs + kTokRows * RS;          // [kTokCols][RS]
   __shared__ double red_d[2][kTokThreads / 32];
   __shared__ unsigned long long red_b[kTokThreads / 32];
   __shared__ uint32_t cnt_tile[2][kTokCols];
-  // query rows of this chunk, all fused heads, as fp32 (transposed)
-  for (int e = threadIdx.x; e < X * kTokRows; e += kTokThreads) {
-    const int r = e / X, x = e % X, h = x / D, d = x % D;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int kVec = 8;                          // bf16 per 16-byte copy
+  const int vecs_per_row = X / kVec;
+  // query rows of this chunk, fused heads side by side
+  for (int e = threadIdx.x; e < kTokRows * vecs_per_row; e += kTokThreads) {
+    const int r = e / vecs_per_row, x = (e % vecs_per_row) * kVec, h = x / D, d = x % D;
     const int u = u0 + r;
-    float val = 0.f;
-    if (u < nt) val = __bfloat162float(p.q[((static_cast<int64_t>(b) * p.H + h) * g.n + i * nt + u) * D + d]);
-    qT[x * kTokRows + r] = val;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (u < nt)
+      val = *reinterpret_cast<const uint4*>(p.q + ((static_cast<int64_t>(b) * p.H + h) * g.n + i * nt + u) * D + d);
+    *reinterpret_cast<uint4*>(qs + r * RS + x) = val;
   }
-  const int ur = (threadIdx.x >> 4) * 2;           // rows ur, ur + 1
-  const int vc = threadIdx.x & 15;                 // columns vc + 16 m
+  const int mr = (warp >> 2) * 16;                 // warp's first tile row
+  const int nc = (warp & 3) * 16;                  // warp's first tile column
   const int v_lo = max(u0 - w, 0), v_hi = min(u0 + kTokRows - 1 + w, nt - 1);
   const double thr = p.pass == 1 ? p.thr[static_cast<int64_t>(b) * F * F + pi] : 0.0;
   const int I0 = (i * nt + u0) / g.block;          // first query block of the chunk
+  // ldmatrix row addresses: A rows mr + (lane % 16), k offset 8 (lane / 16);
+  // B rows nc + 8 (lane / 16) + (lane % 8), k offset 8 ((lane / 8) % 2)
+  const uint32_t a_addr = smem_u32(qs + (mr + (lane & 15)) * RS + ((lane >> 4) << 3));
+  const uint32_t b_addr = smem_u32(ks + (nc + ((lane >> 4) << 3) + (lane & 7)) * RS + (((lane >> 3) & 1) << 3));
+  const int g4 = lane >> 2, t4 = lane & 3;         // accumulator fragment coordinates
   double s1 = 0.0, s2 = 0.0;
   unsigned long long bst = 0ull;
   for (int v0 = v_lo; v0 <= v_hi; v0 += kTokCols) {
-    __syncthreads();   // previous tile's kT and counters are consumed
-    for (int e = threadIdx.x; e < X * kTokCols; e += kTokThreads) {
-      const int c = e / X, x = e % X, h = x / D, d = x % D;
+    __syncthreads();   // previous tile's K rows and counters are consumed
+    for (int e = threadIdx.x; e < kTokCols * vecs_per_row; e += kTokThreads) {
+      const int c = e / vecs_per_row, x = (e % vecs_per_row) * kVec, h = x / D, d = x % D;
       const int v = v0 + c;
-      float val = 0.f;
-      if (v <= v_hi) val = __bfloat162float(p.k[((static_cast<int64_t>(b) * p.H + h) * g.n + j * nt + v) * D + d]);
-      kT[x * kTokCols + c] = val;
+      uint4 val = make_uint4(0u, 0u, 0u, 0u);
+      if (v <= v_hi)
+        val = *reinterpret_cast<const uint4*>(p.k + ((static_cast<int64_t>(b) * p.H + h) * g.n + j * nt + v) * D + d);
+      *reinterpret_cast<uint4*>(ks + c * RS + x) = val;
     }
     if (p.pass == 1 && threadIdx.x < 2 * kTokCols) cnt_tile[threadIdx.x / kTokCols][threadIdx.x % kTokCols] = 0u;
     __syncthreads();
-    float acc[2][4];
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int m = 0; m < 4; ++m) acc[a][m] = 0.f;
-#pragma unroll 8
-    for (int x = 0; x < X; ++x) {
-      const float q0 = qT[x * kTokRows + ur], q1 = qT[x * kTokRows + ur + 1];
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float kv = kT[x * kTokCols + vc + 16 * m];
-        acc[0][m] = fmaf(q0, kv, acc[0][m]);
-        acc[1][m] = fmaf(q1, kv, acc[1][m]);
-      }
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};   // two n8 tiles
+    for (int k0 = 0; k0 < X; k0 += 16) {
+      uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+      ldsm_x4(a_addr + k0 * 2, a0, a1, a2, a3);
+      ldsm_x4(b_addr + k0 * 2, b0, b1, b2, b3);
+      mma_16816(acc[0], a0, a1, a2, a3, b0, b1);
+      mma_16816(acc[1], a0, a1, a2, a3, b2, b3);
     }
 #pragma unroll
-    for (int a = 0; a < 2; ++a) {
-      const int u = u0 + ur + a;
+    for (int nt8 = 0; nt8 < 2; ++nt8) {
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int v = v0 + vc + 16 * m;
+      for (int e = 0; e < 4; ++e) {
+        const int u = u0 + mr + g4 + ((e >> 1) << 3);
+        const int v = v0 + nc + nt8 * 8 + 2 * t4 + (e & 1);
         const int dd = u > v ? u - v : v - u;
         if (u >= nt || v > v_hi || dd > w) continue;
-        const float s = acc[a][m] * p.inv;
+        const float s = acc[nt8][e] * p.inv;
         if (p.pass == 0) {
           s1 += static_cast<double>(s);
           s2 += static_cast<double>(s) * static_cast<double>(s);
@@ -144,7 +173,7 @@ __global__ void __launch_bounds__(kTokThreads) dyntok_tile_kernel(DynTokParams p
           bst = key > bst ? key : bst;
         } else if (static_cast<double>(s) > thr) {
           const int slot = (i * nt + u) / g.block - I0;   // 0 or 1 (a chunk spans at most 2 blocks)
-          atomicAdd(&cnt_tile[slot][vc + 16 * m], 1u);
+          atomicAdd(&cnt_tile[slot][v - v0], 1u);
         }
       }
     }
@@ -160,7 +189,6 @@ __global__ void __launch_bounds__(kTokThreads) dyntok_tile_kernel(DynTokParams p
   }
   if (p.pass == 0) {
     // CTA reduction, then one atomic per quantity
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
       s1 += __shfl_xor_sync(0xffffffffu, s1, off);

@@ -273,7 +273,8 @@ int dynrad_build_sampled_mask(const dynrad_geom *geom, double rho1, double rho2,
  * among equals) is kept.  Pairs at t <= 1 are all kept.  Kept links are
  * aggregated with (theta_c, theta_m) and united with the forced range.
  *
- *   q, k          DEVICE bf16 [B, H, N, D]; D = 64 or 128; hf in [1, min(H, 4)]
+ *   q, k          DEVICE bf16 [B, H, N, D], 16-byte aligned; D = 64 or 128;
+ *                 hf in [1, min(H, 4)]
  *   tau1, tau2    finite z-score thresholds (near / far field)
  *   cand_*, forced_*  from dynrad_build_candidates for geom (DEVICE)
  *   row_ptr       DEVICE int32 [B*H*Nb + 1], rows (b, h, I); every head of a
