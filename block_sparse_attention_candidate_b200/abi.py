@@ -45,6 +45,7 @@ EXPORTED = (
     "dynrad_build_sampled_mask",
     "dynrad_token_mask_workspace_bytes",
     "dynrad_build_token_mask",
+    "dynrad_proxy_error",
 )
 
 
@@ -147,6 +148,8 @@ def lib() -> ctypes.CDLL:
         L.dynrad_build_token_mask.argtypes = [_VP, _VP, _I32, _I32, _I32, _I32, _I32, _GP, ctypes.c_double,
                                               ctypes.c_double, _VP, _VP, _I64, _VP, _VP, _VP, _VP, _I64, _VP, _VP,
                                               _SZ, _VP]
+        L.dynrad_proxy_error.restype = ctypes.c_int
+        L.dynrad_proxy_error.argtypes = [_VP, _VP, _VP, _VP, _I64, _VP, _VP]
         _lib = L
     return _lib
 
@@ -411,3 +414,12 @@ def dynrad_build_token_mask(q, k, geom, cand, tau1, tau2, hf=2, stats=False, str
                                      ctypes.c_void_p(ws.data_ptr() + off), ws_bytes, _stream(stream)),
            "dynrad_build_token_mask")
     return row_ptr, col, st
+
+
+def dynrad_proxy_error(lse_dense, lse_kept, lse2_dense, lse2_kept, stream=None):
+    """(||A_dense - A_masked||_F^2, ||A_dense||_F^2) from four fp32 CUDA LSE vectors."""
+    _require_cuda(lse_dense, lse_kept, lse2_dense, lse2_kept)
+    out = torch.empty(2, dtype=torch.float64, device=lse_dense.device)
+    _check(lib().dynrad_proxy_error(_ptr(lse_dense), _ptr(lse_kept), _ptr(lse2_dense), _ptr(lse2_kept),
+                                    lse_dense.numel(), _ptr(out), _stream(stream)), "dynrad_proxy_error")
+    return out

@@ -201,6 +201,73 @@ __global__ void exp2_diag_kernel(const float* x, float* poly, float* ref, int64_
 
 extern "C" {
 
+}  // extern "C"
+
+namespace {
+
+// Per query row r, from the log-sum-exps of the dense and the masked attention
+// at logit scale c (lse) and 2c (lse2):
+//   sum_j a_j^2 over all keys = exp(lse2_dense - 2 lse_dense),
+//   the same over kept keys   = exp(lse2_kept - 2 lse_dense),
+//   kept mass m               = exp(lse_kept - lse_dense),
+// and the row's squared error between the dense softmax row and the masked,
+// renormalized one: (1 - 1/m)^2 sum_kept a_j^2 + sum_masked a_j^2.
+__global__ void proxy_error_kernel(const float* lse_d, const float* lse_k, const float* lse2_d, const float* lse2_k,
+                                   int64_t n, double* out) {
+  __shared__ double red[2][8];
+  double err = 0.0, tot = 0.0;
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; r < n;
+       r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const double ld = lse_d[r], l2d = lse2_d[r];
+    const double all2 = exp(l2d - 2.0 * ld);
+    double kept2 = 0.0, inv_m = 0.0;
+    if (isfinite(static_cast<double>(lse_k[r]))) {
+      kept2 = exp(static_cast<double>(lse2_k[r]) - 2.0 * ld);
+      inv_m = exp(ld - static_cast<double>(lse_k[r]));
+    }
+    const double f = 1.0 - inv_m;
+    err += (kept2 > 0.0 ? f * f * kept2 : 0.0) + fmax(all2 - kept2, 0.0);
+    tot += all2;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    err += __shfl_xor_sync(0xffffffffu, err, off);
+    tot += __shfl_xor_sync(0xffffffffu, tot, off);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    red[0][warp] = err;
+    red[1][warp] = tot;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double e = 0.0, t = 0.0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
+      e += red[0][w];
+      t += red[1][w];
+    }
+    atomicAdd(out, e);
+    atomicAdd(out + 1, t);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int dynrad_proxy_error(const float* lse_dense, const float* lse_kept, const float* lse2_dense,
+                       const float* lse2_kept, int64_t n, double* out, dynrad_stream_t stream) {
+  if (lse_dense == nullptr || lse_kept == nullptr || lse2_dense == nullptr || lse2_kept == nullptr ||
+      out == nullptr || n < 1)
+    return DYNRAD_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  if (cudaMemsetAsync(out, 0, 2 * sizeof(double), st) != cudaSuccess) return DYNRAD_ERR_CUDA;
+  const int64_t blocks = std::min<int64_t>((n + 255) / 256, 1184);
+  proxy_error_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(lse_dense, lse_kept, lse2_dense, lse2_kept, n,
+                                                                   out);
+  return launch_status();
+}
+
 int dynrad_debug_exp2(const float* x, float* poly_out, float* ref_out, int64_t n, dynrad_stream_t stream) {
   if (x == nullptr || poly_out == nullptr || ref_out == nullptr || n < 0) return DYNRAD_ERR_INVALID_ARG;
   if (n == 0) return DYNRAD_OK;

@@ -244,3 +244,25 @@ def random_qkv_bf16(seed: int, batch: int, heads: int, n: int, dim: int,
     return {t: round_to_bf16_bits(rng.standard_normal((batch, heads, n, dim), dtype=np.float32)
                                   * np.float32(scale))
             for t in _TENSORS}
+
+
+# ---------------------------------------------------------------------------
+# Feature-drift proxy (DynamicRad, Appendix C.2, Eq. 20): the synthetic task the
+# offline parameter search is run on.  This draws the features only; the
+# proxy attention matrix and the objective are computed elsewhere.
+# ---------------------------------------------------------------------------
+DRIFT_REGIMES = {"low": 0.02, "mid": 0.15, "high": 0.40}
+
+
+def ar_features(seed: int, frames: int, tokens_per_frame: int, dim: int, delta: float) -> np.ndarray:
+    """Hidden states h of every token, float32 [frames * tokens_per_frame, dim]:
+    each spatial token position carries its own auto-regressive chain over the
+    frames, h_0 ~ N(0, I), h_t = sqrt(1 - delta^2) h_{t-1} + delta eps_t with
+    eps_t ~ N(0, I) (so every h_t is N(0, I))."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed)))
+    h = np.empty((frames, tokens_per_frame, dim), dtype=np.float64)
+    h[0] = rng.standard_normal((tokens_per_frame, dim))
+    a = math.sqrt(1.0 - delta * delta)
+    for t in range(1, frames):
+        h[t] = a * h[t - 1] + delta * rng.standard_normal((tokens_per_frame, dim))
+    return h.reshape(frames * tokens_per_frame, dim).astype(np.float32)

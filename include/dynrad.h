@@ -374,6 +374,22 @@ int dynrad_host_path(const void *q_host, const void *k_host,
                      size_t workspace_bytes, dynrad_stream_t stream);
 
 /*
+ * Objective of the offline parameter search (Appendix C.4, Eq. 22; no
+ * counterpart on the hot path): from the log-sum-exps of dynrad_sparse_attn
+ * run with a full CSR and with a mask, each at logit scale c and 2c, writes
+ * out[0] = ||A_dense - A_masked||_F^2 and out[1] = ||A_dense||_F^2 over the n
+ * query rows, A the row-softmax matrices (the masked one renormalized over its
+ * kept keys; a row with no kept key is all zero).  Uses, per row,
+ * sum_j a_j^2 = exp(lse(2c) - 2 lse(c)) and kept mass exp(lse_kept - lse_dense).
+ *
+ *   lse_dense, lse_kept, lse2_dense, lse2_kept  DEVICE fp32 [n]
+ *   out           DEVICE double [2] (overwritten)
+ */
+int dynrad_proxy_error(const float *lse_dense, const float *lse_kept,
+                       const float *lse2_dense, const float *lse2_kept,
+                       int64_t n, double *out, dynrad_stream_t stream);
+
+/*
  * Reads the device status word (the first error a kernel recorded since the
  * last clear) into *status_out; clears it when clear != 0.  SYNCHRONIZES the
  * stream.  Returns DYNRAD_ERR_CUDA if the stream itself reports an error.

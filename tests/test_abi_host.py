@@ -245,3 +245,11 @@ def test_token_mask_argument_errors_before_launch():
     # token) link counters; kept lists, per-batch CSR, scan partials
     base = 2 * F * F * 32 + 2 * nb * n * 4 + 2 * 100 * 4 * 2 + (2 * nb + 1) * 4 + 8
     assert base <= need < base + 256 * 9
+
+
+def test_proxy_error_argument_errors():
+    L = abi.lib()
+    p = ctypes.c_void_p(0x10000)
+    assert L.dynrad_proxy_error(None, p, p, p, 10, p, None) == abi.DYNRAD_ERR_INVALID_ARG
+    assert L.dynrad_proxy_error(p, p, p, p, 0, p, None) == abi.DYNRAD_ERR_INVALID_ARG
+    assert L.dynrad_proxy_error(p, p, p, p, 10, None, None) == abi.DYNRAD_ERR_INVALID_ARG
