@@ -21,7 +21,11 @@ from "DynamicRad: Content-Adaptive Sparse Attention for Long Video Diffusion"
 * ``dynamic_tokens`` -- the paper-exact dynamic-threshold mode of Sec. 3.2
   (Eqs. 9-11, Eq. 19): fused-head proxy logits on the candidate token pairs,
   per-frame-pair z-scores, tau_1 / tau_2 thresholds with the top-pair
-  fallback, aggregated to blocks.
+  fallback, aggregated to blocks;
+* ``backward``  -- gradients dQ, dK, dV of the block-masked attention (for the
+  mask-aware fine-tuning of Sec. 3.3);
+* ``proxy``     -- the objective of the offline parameter search on the
+  feature-drift proxy (Appendix C.2-C.4, Eq. 22).
 
 Every function is pinned by ``-m "not gpu"`` tests to closed forms, library
 routines for special cases, brute force on tiny inputs, or invariants the
