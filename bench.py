@@ -256,6 +256,8 @@ def main():
     ap.add_argument("--token-tau", default="0.0,1.0", help="tau_1,tau_2 of the token-level dynamic mode")
     ap.add_argument("--token-theta", default="0.2,0.5",
                     help="theta_c,theta_m (block aggregation) of the token-level dynamic mode")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the attention backward (dQ, dK, dV under the selected mask) measurement")
     ap.add_argument("--e2e-chunk", type=int, default=4,
                     help="(batch, head) rows per chunk of the end-to-end host path")
     ap.add_argument("--no-dense", action="store_true")
@@ -504,6 +506,41 @@ def main():
                  "speedup_vs_dense": round(dense["ms"] / attn_t, 2) if dense else None}
         del rp_t, col_t, o_t, lse_t
 
+    # ---- backward of the attention under the first run's selected mask (the
+    # gradient the mask-aware fine-tuning trains through), dO seeded N(0, 1)
+    backward = None
+    if not args.no_backward:
+        r0 = runs[0]
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(2027)
+        dout = torch.randn(q.shape, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        grads = tuple(torch.empty_like(q) for _ in range(3))
+        rp0, col0 = r0["sel"].row_ptr, r0["sel"].col_idx
+        bws = torch.empty(abi.lib().dynrad_attn_backward_workspace_bytes(B, H, N, r0["geom"].block, col0.numel()),
+                          dtype=torch.uint8, device=dev)
+        run_path(r0, q, k, v)
+        for _ in range(2):
+            abi.dynrad_attn_backward(q, k, v, r0["o"], r0["lse"], dout, r0["geom"].block, rp0, col0,
+                                     grads=grads, workspace=bws)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        reps = 3
+        e0.record(stream)
+        for _ in range(reps):
+            abi.dynrad_attn_backward(q, k, v, r0["o"], r0["lse"], dout, r0["geom"].block, rp0, col0,
+                                     grads=grads, workspace=bws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        st = abi.dynrad_device_status(clear=True)
+        if st != 0:
+            raise RuntimeError(f"device status after the backward run: {abi.status_string(st)}")
+        bwd_ms = e0.elapsed_time(e1) / reps
+        # algorithmic backward FLOPs: S, dP, dV, dQ, dK products, 2.5x the forward's
+        bflops = 2.5 * flops_run[0]
+        backward = {"run": r0["label"], "ms": round(bwd_ms, 3), "tflops": round(bflops / (bwd_ms * 1e-3) / 1e12, 1),
+                    "fwd_attn_ms": run_info[r0["label"]]["attn_ms"], "flop_model": "10 * D per kept (query, key)"}
+        del dout, grads, bws
+
     # ---- end to end through the host-memory entry point: pinned host Q, K, V
     # in, every run's O and LSE back to pinned host memory, the copies
     # overlapped with the kernels by dynrad_host_path (chunks of heads)
@@ -574,6 +611,7 @@ def main():
         "dense_same_kernel": dense,
         "sampled_static": sampled,
         "token_dynamic": token,
+        "backward": backward,
         "stage_ms_per_step": {"candidates": round(float(stage_ms[:, 0].sum()), 4),
                               "selection": round(float(stage_ms[:, 1].sum()), 4),
                               "attention": round(attn_ms_total, 4)},

@@ -46,6 +46,8 @@ EXPORTED = (
     "dynrad_token_mask_workspace_bytes",
     "dynrad_build_token_mask",
     "dynrad_proxy_error",
+    "dynrad_attn_backward_workspace_bytes",
+    "dynrad_attn_backward",
 )
 
 
@@ -150,6 +152,11 @@ def lib() -> ctypes.CDLL:
                                               _SZ, _VP]
         L.dynrad_proxy_error.restype = ctypes.c_int
         L.dynrad_proxy_error.argtypes = [_VP, _VP, _VP, _VP, _I64, _VP, _VP]
+        L.dynrad_attn_backward_workspace_bytes.restype = _SZ
+        L.dynrad_attn_backward_workspace_bytes.argtypes = [_I32, _I32, _I32, _I32, _I64]
+        L.dynrad_attn_backward.restype = ctypes.c_int
+        L.dynrad_attn_backward.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _I32, _I32, _I32, _I32, _I32, _VP, _VP,
+                                           _I64, ctypes.c_float, _VP, _VP, _VP, _VP, _SZ, _VP]
         _lib = L
     return _lib
 
@@ -278,6 +285,26 @@ def dynrad_sparse_attn(q, k, v, block, row_ptr, col_idx, scale=0.0, out=None, ls
                                     _ptr(col_idx), float(scale), _ptr(o), _ptr(lse_t), _stream(stream)),
            "dynrad_sparse_attn")
     return o, lse_t
+
+
+def dynrad_attn_backward(q, k, v, o, lse, dout, block, row_ptr, col_idx, scale=0.0, grads=None, workspace=None,
+                         stream=None):
+    """Gradient of stage 3 under the same CSR.  q, k, v, o, dout: bf16
+    [B, H, N, D] CUDA; lse fp32 [B, H, N] from dynrad_sparse_attn.
+    Returns (dq, dk, dv), bf16 [B, H, N, D]."""
+    _require_cuda(q, k, v, o, lse, dout, row_ptr, col_idx)
+    B, H, N, D = q.shape
+    dq, dk, dv = grads if grads is not None else tuple(torch.empty_like(q) for _ in range(3))
+    cap = col_idx.numel()
+    L = lib()
+    need = L.dynrad_attn_backward_workspace_bytes(B, H, N, int(block), cap)
+    if need == 0:
+        raise DynradError(1, "dynrad_attn_backward_workspace_bytes")
+    ws = torch.empty(need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    _check(L.dynrad_attn_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), B, H, N, D, int(block),
+                                  _ptr(row_ptr), _ptr(col_idx), cap, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
+                                  _ptr(ws), ws.numel(), _stream(stream)), "dynrad_attn_backward")
+    return dq, dk, dv
 
 
 def dynrad_select_blocks_static_scratch(q, k, geom, cand, mode, value, row_ptr, col_idx, scores=None,

@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libdynrad.so")
 SOURCES = ["dynrad.cu", "host_path.cu"]
-HEADERS = ["common.cuh", "candidates.cuh", "select.cuh", "attention.cuh", "sampling.cuh", "dyntok.cuh"]
+HEADERS = ["common.cuh", "candidates.cuh", "select.cuh", "attention.cuh", "sampling.cuh", "dyntok.cuh", "backward.cuh", "warp_mma.cuh"]
 
 
 def nvcc_path() -> str:

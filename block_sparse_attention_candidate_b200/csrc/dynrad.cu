@@ -15,6 +15,7 @@
 #include "attention.cuh"
 #include "candidates.cuh"
 #include "common.cuh"
+#include "backward.cuh"
 #include "dyntok.cuh"
 #include "sampling.cuh"
 #include "select.cuh"
@@ -716,6 +717,134 @@ int dynrad_build_token_mask(const void* q, const void* k, int32_t B, int32_t H, 
     if ((rc = launch_status()) != DYNRAD_OK) return rc;
   }
   return DYNRAD_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+struct BwdWorkspace {
+  size_t rowdot, t_ptr, t_col, partial, total;
+};
+
+BwdWorkspace bwd_layout(int64_t bh, int64_t n, int64_t nb, int64_t col_cap) {
+  BwdWorkspace w;
+  const int64_t rows = bh * nb;
+  const int64_t tiles = (rows + 1 + kScanTile - 1) / kScanTile;
+  w.rowdot = 0;
+  w.t_ptr = align256(w.rowdot + static_cast<size_t>(bh * n) * 4);
+  w.t_col = align256(w.t_ptr + static_cast<size_t>(rows + 1) * 4);
+  w.partial = align256(w.t_col + static_cast<size_t>(col_cap) * 4);
+  w.total = align256(w.partial + static_cast<size_t>(tiles) * 8);
+  return w;
+}
+
+template <int D>
+int launch_backward(const BwdParams& bp, cudaStream_t st) {
+  const size_t smem = static_cast<size_t>(4) * kBwdTile * (D + 8) * 2;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess ||
+        cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return DYNRAD_ERR_CUDA;
+    attr = true;
+  }
+  const dim3 grid((bp.N + kBwdTile - 1) / kBwdTile, bp.BH);
+  bwd_dkv_kernel<D><<<grid, kBwdThreads, smem, st>>>(bp);
+  int rc = launch_status();
+  if (rc != DYNRAD_OK) return rc;
+  bwd_dq_kernel<D><<<grid, kBwdThreads, smem, st>>>(bp);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dynrad_attn_backward_workspace_bytes(int32_t B, int32_t H, int32_t N, int32_t block, int64_t col_cap) {
+  if (B < 1 || H < 1 || N < 1 || block < 1 || col_cap < 0) return 0;
+  const int64_t nb = (static_cast<int64_t>(N) + block - 1) / block;
+  return bwd_layout(static_cast<int64_t>(B) * H, N, nb, col_cap).total;
+}
+
+int dynrad_attn_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                         const float* lse, int32_t B, int32_t H, int32_t N, int32_t D, int32_t block,
+                         const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap, float scale, void* dq,
+                         void* dk, void* dv, void* workspace, size_t workspace_bytes, dynrad_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || dout == nullptr || lse == nullptr ||
+      row_ptr == nullptr || col_idx == nullptr || dq == nullptr || dk == nullptr || dv == nullptr ||
+      workspace == nullptr)
+    return DYNRAD_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1 || col_cap < 0) return DYNRAD_ERR_INVALID_ARG;
+  if (!(scale >= 0.0f) || !std::isfinite(scale)) return DYNRAD_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return DYNRAD_ERR_UNSUPPORTED;
+  if (block != 64 && block != 128) return DYNRAD_ERR_UNSUPPORTED;
+  for (const void* ptr : {q, k, v, o, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                          static_cast<const void*>(dv)})
+    if (!aligned16(ptr)) return DYNRAD_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DYNRAD_ERR_INVALID_ARG;
+  const int64_t bh = static_cast<int64_t>(B) * H;
+  if (bh > 65535) return DYNRAD_ERR_UNSUPPORTED;
+  const int64_t nb = (static_cast<int64_t>(N) + block - 1) / block;
+  if (bh * nb + 1 > INT32_MAX) return DYNRAD_ERR_UNSUPPORTED;
+  const BwdWorkspace w = bwd_layout(bh, N, nb, col_cap);
+  if (workspace_bytes < w.total) return DYNRAD_ERR_CAPACITY;
+  cudaStream_t st = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  BwdParams bp;
+  bp.q = static_cast<const __nv_bfloat16*>(q);
+  bp.k = static_cast<const __nv_bfloat16*>(k);
+  bp.v = static_cast<const __nv_bfloat16*>(v);
+  bp.o = static_cast<const __nv_bfloat16*>(o);
+  bp.dout = static_cast<const __nv_bfloat16*>(dout);
+  bp.lse = lse;
+  bp.rowdot = reinterpret_cast<float*>(ws + w.rowdot);
+  bp.row_ptr = row_ptr;
+  bp.col_idx = col_idx;
+  bp.t_ptr = reinterpret_cast<int32_t*>(ws + w.t_ptr);
+  bp.t_col = reinterpret_cast<int32_t*>(ws + w.t_col);
+  bp.t_cap = col_cap;
+  bp.dq = static_cast<__nv_bfloat16*>(dq);
+  bp.dk = static_cast<__nv_bfloat16*>(dk);
+  bp.dv = static_cast<__nv_bfloat16*>(dv);
+  bp.BH = static_cast<int>(bh);
+  bp.N = N;
+  bp.nb = static_cast<int>(nb);
+  bp.block = block;
+  bp.scale = scale == 0.0f ? 1.0f / std::sqrt(static_cast<float>(D)) : scale;
+  int rc;
+  const int64_t rows = bh * nb;
+  // D_r, then the transposed CSR
+  const int64_t nrows = bh * N;
+  bwd_rowdot_kernel<<<static_cast<unsigned>((nrows * 32 + 255) / 256), 256, 0, st>>>(bp, D);
+  if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  if (cudaMemsetAsync(bp.t_ptr, 0, static_cast<size_t>(rows + 1) * 4, st) != cudaSuccess) return DYNRAD_ERR_CUDA;
+  const unsigned wblocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+  bwd_tcount_kernel<<<wblocks, 256, 0, st>>>(bp);
+  if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  {
+    int64_t* partial = reinterpret_cast<int64_t*>(ws + w.partial);
+    const int64_t tiles = (rows + 1 + kScanTile - 1) / kScanTile;
+    scan_partial_kernel<<<static_cast<unsigned>(tiles), kScanThreads, 0, st>>>(bp.t_ptr, rows, partial);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+    CompactParams cp;
+    cp.row_ptr = bp.t_ptr;
+    cp.partial = partial;
+    cp.rows = rows;
+    cp.nb = static_cast<int>(nb);
+    cp.cand_row_ptr = nullptr;
+    cp.kept_tmp = nullptr;
+    cp.cand_nnz = 0;
+    cp.col_idx = nullptr;
+    cp.col_cap = 0;
+    scan_apply_kernel<<<static_cast<unsigned>(tiles), kScanThreads, 0, st>>>(cp);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  }
+  bwd_tfill_kernel<<<wblocks, 256, 0, st>>>(bp);
+  if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  return D == 128 ? launch_backward<128>(bp, st) : launch_backward<64>(bp, st);
 }
 
 int dynrad_sparse_attn(const void* q, const void* k, const void* v, int32_t B, int32_t H, int32_t N,

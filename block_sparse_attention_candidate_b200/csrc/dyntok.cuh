@@ -29,6 +29,7 @@
 
 #include "candidates.cuh"
 #include "common.cuh"
+#include "warp_mma.cuh"
 
 namespace dynrad {
 
@@ -71,22 +72,6 @@ __device__ __forceinline__ float tok_key_to_float(uint32_t key) {
 // Row stride (bf16 elements) of the staged Q / K rows: 8 elements of padding
 // keep the 8 rows an ldmatrix reads in distinct bank groups.
 __host__ __device__ constexpr int tok_row_stride(int x) { return x + 8; }
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-// D += A(16x16, row) B(16x8, col), bf16 inputs, fp32 accumulation.
-__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                          uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 // The logit tiles are dense 32 x 64 x (H_f * D) products: warp-level bf16
 // tensor-core MMAs (m16n8k16, fp32 accumulation) on Q / K rows staged in shared

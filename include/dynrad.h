@@ -14,6 +14,7 @@
  *      tau).  Output: CSR block indices.
  *   3. dynrad_sparse_attn      -- block-sparse softmax attention over the kept
  *      blocks, Eqs. 12-13 with epsilon -> 0, returning O and the log-sum-exp.
+ *      dynrad_attn_backward is its gradient (dQ, dK, dV) under the same mask.
  *
  * Conventions shared by every call
  *   - Pointers named q, k, v, o, lse, *_row_ptr, *_col*, forced_*, scores_out,
@@ -388,6 +389,43 @@ int dynrad_host_path(const void *q_host, const void *k_host,
 int dynrad_proxy_error(const float *lse_dense, const float *lse_kept,
                        const float *lse2_dense, const float *lse2_kept,
                        int64_t n, double *out, dynrad_stream_t stream);
+
+/*
+ * Backward of stage 3 (the gradient that the mask-aware fine-tuning of
+ * Sec. 3.3 trains through): given dO, the forward's O and LSE and the SAME
+ * kept-block CSR, computes for every (b, h)
+ *   P_qk  = exp(scale * q.k - lse_q) on the kept blocks' valid keys, else 0
+ *   D_q   = sum_d dO_qd O_qd
+ *   dV_k  = sum_q P_qk dO_q
+ *   dS_qk = P_qk (dO_q . v_k - D_q)
+ *   dQ_q  = scale * sum_k dS_qk k_k,   dK_k = scale * sum_q dS_qk q_q
+ * (the exact gradient of the forward's output; keys of unkept blocks get
+ * dK = dV = 0, rows with no kept block get dQ = 0).  Warp-level bf16 tensor
+ * core products with fp32 accumulation; no atomics (one CTA owns each 64-row
+ * tile of dK/dV and of dQ).  The workspace holds D_q and the transposed CSR.
+ *
+ *   q, k, v, o, dout  device bf16 [B, H, N, D], D = 64 or 128
+ *   lse           device fp32 [B, H, N] (the forward's, natural log)
+ *   block         64 or 128
+ *   row_ptr, col_idx  the forward's CSR (device int32, B*H*Nb rows, strictly
+ *                 ascending block indices in [0, Nb) per row)
+ *   col_cap       capacity of the transposed CSR: >= row_ptr[B*H*Nb]
+ *                 (overflow is flagged in the device status)
+ *   scale         logit scale; 0 means 1/sqrt(D)
+ *   dq, dk, dv    device bf16 [B, H, N, D] (overwritten)
+ *   workspace     device, 256-byte aligned, workspace_bytes >=
+ *                 dynrad_attn_backward_workspace_bytes(B, H, N, block, col_cap)
+ *   B * H <= 65535.
+ */
+size_t dynrad_attn_backward_workspace_bytes(int32_t B, int32_t H, int32_t N,
+                                            int32_t block, int64_t col_cap);
+int dynrad_attn_backward(const void *q, const void *k, const void *v,
+                         const void *o, const void *dout, const float *lse,
+                         int32_t B, int32_t H, int32_t N, int32_t D,
+                         int32_t block, const int32_t *row_ptr,
+                         const int32_t *col_idx, int64_t col_cap, float scale,
+                         void *dq, void *dk, void *dv, void *workspace,
+                         size_t workspace_bytes, dynrad_stream_t stream);
 
 /*
  * Reads the device status word (the first error a kernel recorded since the

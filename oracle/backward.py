@@ -44,3 +44,47 @@ def sparse_attention_backward(q, k, v, do, block: int, row_ptr, col, scale=None)
     dq = scale * (ds @ k)
     dk = scale * (ds.T @ q)
     return dq, dk, dv, o
+
+
+def _block_tokens(block: int, n: int, blocks) -> np.ndarray:
+    parts = [np.arange(b * block, min((b + 1) * block, n), dtype=np.int64) for b in blocks]
+    return np.concatenate(parts) if parts else np.zeros(0, dtype=np.int64)
+
+
+def query_block_backward(q, k, v, do, block: int, kept, i: int, scale=None):
+    """The same gradients restricted to the query tokens of block i, whose kept
+    key blocks are `kept` (for sampled checks at sizes where the [N, N] mask
+    does not fit).  Returns (rows, keys, p, ds, dq_rows): the query and key
+    token indices, P and dS over [rows, keys], and dQ of the rows."""
+    n, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    rows = np.arange(i * block, min((i + 1) * block, n), dtype=np.int64)
+    keys = _block_tokens(block, n, kept)
+    if len(keys) == 0:
+        z = np.zeros((len(rows), 0))
+        return rows, keys, z, z, np.zeros((len(rows), d))
+    p = masked_softmax(scale * (q[rows] @ k[keys].T), np.ones((len(rows), len(keys)), dtype=bool))
+    dp = do[rows] @ v[keys].T
+    ds = p * (dp - (dp * p).sum(axis=1, keepdims=True))
+    return rows, keys, p, ds, scale * (ds @ k[keys])
+
+
+def key_block_backward(q, k, v, do, block: int, row_ptr, col, j: int, scale=None):
+    """dK, dV of the key tokens of block j: the sum over every query block that
+    keeps j of that block's P^T dO and scale dS^T Q on j's keys, each query
+    row normalised over its own kept keys.  Returns (keys_j, dk_j, dv_j)."""
+    n, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    keys_j = _block_tokens(block, n, [j])
+    dk = np.zeros((len(keys_j), d))
+    dv = np.zeros((len(keys_j), d))
+    nb = -(-n // block)
+    for i in range(nb):
+        kept = np.asarray(col[int(row_ptr[i]):int(row_ptr[i + 1])], dtype=np.int64)
+        if not np.any(kept == j):
+            continue
+        rows, keys, p, ds, _ = query_block_backward(q, k, v, do, block, kept, i, scale)
+        sel = np.searchsorted(keys, keys_j)
+        dv += p[:, sel].T @ do[rows]
+        dk += scale * (ds[:, sel].T @ q[rows])
+    return keys_j, dk, dv

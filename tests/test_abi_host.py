@@ -253,3 +253,41 @@ def test_proxy_error_argument_errors():
     assert L.dynrad_proxy_error(None, p, p, p, 10, p, None) == abi.DYNRAD_ERR_INVALID_ARG
     assert L.dynrad_proxy_error(p, p, p, p, 0, p, None) == abi.DYNRAD_ERR_INVALID_ARG
     assert L.dynrad_proxy_error(p, p, p, p, 10, None, None) == abi.DYNRAD_ERR_INVALID_ARG
+
+
+def test_backward_argument_errors_before_launch():
+    L = abi.lib()
+    p = ctypes.c_void_p(0x10000)
+    ws = ctypes.c_void_p(0x100000)
+
+    def call(**kw):
+        a = dict(q=p, B=1, H=2, N=300, D=128, block=64, cap=100, scale=0.0, dq=p, ws=ws, ws_bytes=1 << 40)
+        a.update(kw)
+        return L.dynrad_attn_backward(a["q"], p, p, p, p, p, a["B"], a["H"], a["N"], a["D"], a["block"], p, p,
+                                      a["cap"], a["scale"], a["dq"], p, p, a["ws"], a["ws_bytes"], None)
+
+    assert call(q=None) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(dq=None) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(N=0) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(cap=-1) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(scale=-0.5) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == abi.DYNRAD_ERR_INVALID_ARG
+    assert call(D=96) == abi.DYNRAD_ERR_UNSUPPORTED
+    assert call(block=32) == abi.DYNRAD_ERR_UNSUPPORTED
+    assert call(dq=ctypes.c_void_p(0x10008)) == abi.DYNRAD_ERR_INVALID_ARG    # not 16-byte aligned
+    assert call(ws=ctypes.c_void_p(0x100010)) == abi.DYNRAD_ERR_INVALID_ARG   # not 256-byte aligned
+    assert call(B=300, H=300) == abi.DYNRAD_ERR_UNSUPPORTED                   # B*H > 65535
+    assert call(ws_bytes=1024) == abi.DYNRAD_ERR_CAPACITY
+
+
+def test_backward_workspace_size_formula():
+    L = abi.lib()
+    B, H, N, block, cap = 1, 40, 75600, 64, 11_000_000
+    nb = -(-N // block)
+    rows = B * H * nb
+    tiles = -(-(rows + 1) // 2048)
+    got = L.dynrad_attn_backward_workspace_bytes(B, H, N, block, cap)
+    # D_r per query row (fp32), transposed CSR offsets and entries (int32), scan partials
+    need = B * H * N * 4 + (rows + 1) * 4 + cap * 4 + tiles * 8
+    assert need <= got < need + 4 * 256
+    assert L.dynrad_attn_backward_workspace_bytes(0, H, N, block, cap) == 0

@@ -75,3 +75,25 @@ def test_softmax_gradient_identity():
     o = p @ v
     dp = do @ v.T
     np.testing.assert_allclose((dp * p).sum(axis=1), (do * o).sum(axis=1), atol=1e-12)
+
+
+def test_block_restricted_forms_match_the_full_backward():
+    rng = np.random.default_rng(3)
+    n, d, block = 45, 5, 8                        # ragged last block
+    q, k, v, do = (rng.standard_normal((n, d)) for _ in range(4))
+    nb = -(-n // block)
+    keep = rng.random((nb, nb)) < 0.45
+    keep[2, :] = False                            # a row with no kept block
+    keep[:, 4] = False                            # a key block nobody keeps
+    keep[0, 4] = True                             # ... except query block 0
+    keep[:, 3] = False                            # a key block nobody keeps at all
+    rp, col = _csr(keep)
+    dq, dk, dv, _ = OB.sparse_attention_backward(q, k, v, do, block, rp, col, scale=0.7)
+    for i in range(nb):
+        rows, _, _, _, dq_i = OB.query_block_backward(q, k, v, do, block, col[rp[i]:rp[i + 1]], i, scale=0.7)
+        np.testing.assert_allclose(dq_i, dq[rows], atol=1e-12)
+    for j in range(nb):
+        keys, dk_j, dv_j = OB.key_block_backward(q, k, v, do, block, rp, col, j, scale=0.7)
+        np.testing.assert_allclose(dk_j, dk[keys], atol=1e-12)
+        np.testing.assert_allclose(dv_j, dv[keys], atol=1e-12)
+    assert np.all(dk[24:32] == 0) and np.all(dv[24:32] == 0)
