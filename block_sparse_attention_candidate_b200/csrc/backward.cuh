@@ -6,30 +6,20 @@
 //   dV = P^T dO,  dP = dO V^T,  dS = P (dP - D_r),  D_r = rowsum(dO * O),
 //   dQ = scale dS K,  dK = scale dS^T Q.
 //
-// Kernels (64-row tiles; a block of 64 or 128 tokens is one or two tiles; the
-// tiles' products are warp-level bf16 tensor-core MMAs, m16n8k16 with fp32
-// accumulation, each warp owning 16 rows of its CTA's tile):
+// Kernels:
 //   bwd_rowdot_kernel     D_r per query row.
 //   bwd_tcount_kernel, scan, bwd_tfill_kernel   the transposed CSR: for each
 //                         key block, the query blocks that keep it, ascending.
-//   bwd_dkv_kernel<D>     one CTA per (head, 64-key tile): walks the key
-//                         block's query blocks, recomputes S^T and dP^T, and
-//                         accumulates dV and dK in registers (no atomics).
-//   bwd_dq_kernel<D>      one CTA per (head, 64-query tile): walks the row's
-//                         kept key blocks and accumulates dQ (no atomics).
-// P^T / dS^T feed the second products straight from the accumulator
-// registers (the m16n8 accumulator pairs are the m16k16 operand pairs).
+//   bwd_tc_kernel<D, BS, true>   dK, dV per 128-key tile (tcgen05, TMEM, TMA).
+//   bwd_tc_kernel<D, BS, false>  dQ per 128-query tile.
+// Each output row is owned by one CTA: no atomics, deterministic.
 #pragma once
 
 #include <cuda_bf16.h>
 
 #include "common.cuh"
-#include "warp_mma.cuh"
 
 namespace dynrad {
-
-constexpr int kBwdTile = 64;
-constexpr int kBwdThreads = 128;
 
 struct BwdParams {
   const __nv_bfloat16* q;
@@ -111,202 +101,409 @@ __global__ void bwd_tfill_kernel(BwdParams p) {
   }
 }
 
-// Stage 64 rows x D of a [BH, N, D] bf16 tensor into shared memory (row
-// stride D + 8), zeros past N.
-template <int D>
-__device__ __forceinline__ void bwd_stage(__nv_bfloat16* dst, const __nv_bfloat16* src, int64_t bh, int N, int r0) {
-  constexpr int kVec = D / 8;   // 16-byte pieces per row
-  for (int e = threadIdx.x; e < kBwdTile * kVec; e += kBwdThreads) {
-    const int r = e / kVec, x = (e % kVec) * 8;
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (r0 + r < N) val = *reinterpret_cast<const uint4*>(src + (bh * N + r0 + r) * D + x);
-    *reinterpret_cast<uint4*>(dst + r * (D + 8) + x) = val;
-  }
-}
 
-// acc[8][4] (16 rows x 64 columns) += A(16 x D rows of a_s) * B^T, B = 64 rows x D of b_s
-template <int D>
-__device__ __forceinline__ void bwd_rows_by_rows(float (&acc)[8][4], const __nv_bfloat16* a_s, const __nv_bfloat16* b_s,
-                                                 int row0, int lane) {
-  constexpr int RS = D + 8;
-  const uint32_t a_addr = smem_u32(a_s + (row0 + (lane & 15)) * RS + ((lane >> 4) << 3));
-  const uint32_t b_addr = smem_u32(b_s + (((lane >> 4) << 3) + (lane & 7)) * RS + (((lane >> 3) & 1) << 3));
-#pragma unroll
-  for (int k0 = 0; k0 < D; k0 += 16) {
-    uint32_t a0, a1, a2, a3;
-    ldsm_x4(a_addr + k0 * 2, a0, a1, a2, a3);
-#pragma unroll
-    for (int np = 0; np < 4; ++np) {
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4(b_addr + (np * 16 * RS + k0) * 2, b0, b1, b2, b3);
-      mma_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
-      mma_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+// ----------------------------------------------------------------------------
+// Tensor-core gradient kernels.  One template serves both sides:
+//   KV = true   one CTA per (head, 128-key tile): resident K, V; streams the
+//               Q / dO rows of the query blocks that keep the tile's key
+//               blocks; accumulates dV = P^T dO and dK = dS^T Q.
+//   KV = false  one CTA per (head, 128-query tile): resident Q, dO; streams the
+//               K / V rows of the tile's kept key blocks; accumulates dQ = dS K.
+// The tile's rows are R = 128 / BS blocks; their lists (transposed CSR for
+// KV, the forward's CSR otherwise) are merged into one ascending walk, and a
+// union member's BS rows are streamed as BS / 64 steps of 64 rows.  A step's
+// mask bit r says whether list r holds the member: the tile rows of block r
+// get P = 0 otherwise.
+//
+// Per step j (buffer b = j & 1):
+//   G12  X_b = A0 B0^T, Y_b = A1 B1^T (A = resident tiles, B = the step's
+//        tiles; M = 128, N = 64, K = D).  KV: X = S^T, Y = dP^T; else X = S,
+//        Y = dP.
+//   elementwise (warps 0-3, thread = TMEM lane = tile row): P = 2^(X c - lse2),
+//        dS = P (Y - D_r); P (KV only) and dS are written back as bf16 pairs
+//        over the first 32 columns of X_b and Y_b.
+//   G34  KV: dV += P^T B1, dK += dS^T B0; else dQ += dS B0 (A from tensor
+//        memory, B = the step's tile as the MN-major operand; M = 128, N = D,
+//        K = 64).
+// The MMA thread issues G34(j) and then G12(j + 2) into the same buffer, so
+// the tensor core overlaps step j + 1's G12 with step j's elementwise work.
+//
+// Warp roles (192 threads): warps 0-3 elementwise and epilogue, warp 4
+// producer (list walk, TMA loads into a ring of slots, per-query lse2 / D_r of
+// the step for KV), warp 5 MMA issuer.  Tensor memory (512 columns): acc0 at 0
+// (dV or dQ), acc1 at D (dK), X_b at 2D' + 64 b, Y_b at 2D' + 128 + 64 b with
+// D' = D for KV and D / 2 otherwise.  Every wait is bounded (common.cuh).
+// ----------------------------------------------------------------------------
+struct BwdStepMeta {
+  int32_t row0;     // first streamed row of the step
+  uint32_t mask;    // bit r: list r holds the union member
+  int32_t end;      // 1: the walk is over
+  int32_t pad;
+};
+
+template <int D, int BS, bool KV>
+struct BwdTcCfg {
+  static constexpr int kRows = 128;
+  static constexpr int kStep = 64;
+  static constexpr int kR = kRows / BS;
+  static constexpr int kSPB = BS / kStep;
+  static constexpr int kChunks = D / 64;
+  static constexpr int kResBytes = kRows * D * 2;
+  static constexpr int kResChunk = kRows * 128;
+  static constexpr int kStepBytes = kStep * D * 2;
+  static constexpr int kStepChunk = kStep * 128;
+  static constexpr int kSlotBytes = 2 * kStepBytes + 1024;   // two tiles, lse2 / D_r / meta
+  static constexpr int kSmemCtrl = 1024;
+  static constexpr int kBudget = 227 * 1024 - kSmemCtrl - 1024;
+  static constexpr int kSlotsRaw = (kBudget - 2 * kResBytes) / kSlotBytes;
+  static constexpr int kSlots = kSlotsRaw > 6 ? 6 : kSlotsRaw;
+  static constexpr int kSmemData = 2 * kResBytes + kSlots * kSlotBytes;
+  static constexpr int kSmemTotal = kSmemData + kSmemCtrl + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kAcc0 = 0;
+  static constexpr uint32_t kAcc1 = D;
+  static constexpr uint32_t kXY = KV ? 2 * D : D;
+  __host__ __device__ static constexpr uint32_t col_x(int b) { return kXY + 64u * b; }
+  __host__ __device__ static constexpr uint32_t col_y(int b) { return kXY + 128u + 64u * b; }
+  static_assert(D == 64 || D == 128, "head dim");
+  static_assert(BS == 64 || BS == 128, "block size");
+  static_assert(kSlots >= 3, "the MMA issue order needs three slots");
+  static_assert(kXY + 256 <= kTmemCols, "tensor memory");
+  static_assert(kSmemTotal <= 227 * 1024, "shared memory");
+};
+
+template <int D, int BS, bool KV>
+__global__ void __launch_bounds__(192, 1)
+    bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_res0, const __grid_constant__ CUtensorMap tm_res1,
+                  const __grid_constant__ CUtensorMap tm_step0, const __grid_constant__ CUtensorMap tm_step1,
+                  const BwdParams p) {
+  using C = BwdTcCfg<D, BS, KV>;
+  constexpr int NS = C::kSlots;
+  extern __shared__ uint8_t bwd_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(bwd_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* res_smem = smem;                        // A0 at 0, A1 at kResBytes
+  uint8_t* slot_smem = smem + 2 * C::kResBytes;    // step j in slot j % NS
+  uint8_t* ctrl = smem + C::kSmemData;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(ctrl);
+  uint64_t* res_full = bar;
+  uint64_t* slot_full = bar + 1;          // [NS]
+  uint64_t* slot_empty = slot_full + NS;  // [NS]
+  uint64_t* s_full = slot_empty + NS;     // [2]
+  uint64_t* p_full = s_full + 2;          // [2]
+  uint64_t* drain = p_full + 2;
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_s + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const int tile0 = blockIdx.x * C::kRows;   // first resident row
+  const int blk0 = blockIdx.x * C::kR;       // first resident block
+  const int nb = p.nb;
+  const float log2e = 1.4426950408889634f;
+
+  auto slot_tile = [&](int j, int t) -> uint8_t* { return slot_smem + (j % NS) * C::kSlotBytes + t * C::kStepBytes; };
+  auto slot_tail = [&](int j) -> uint8_t* { return slot_smem + (j % NS) * C::kSlotBytes + 2 * C::kStepBytes; };
+
+  if (threadIdx.x == 0) {
+    mbar_init(res_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&slot_full[s], 32);
+      mbar_init(&slot_empty[s], 1);
     }
-  }
-}
-
-// out[D/8][4] (16 rows x D) += X (16 x 64, from accumulator registers) * B, B = 64 rows x D of b_s
-template <int D>
-__device__ __forceinline__ void bwd_acc_times_rows(float (&out)[D / 8][4], const float (&x)[8][4],
-                                                   const __nv_bfloat16* b_s, int lane) {
-  constexpr int RS = D + 8;
-  const uint32_t b_addr = smem_u32(b_s + ((((lane >> 3) & 1) << 3) + (lane & 7)) * RS + ((lane >> 4) << 3));
-#pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
-    const uint32_t a0 = pack_bf16x2(x[2 * kk][0], x[2 * kk][1]);
-    const uint32_t a1 = pack_bf16x2(x[2 * kk][2], x[2 * kk][3]);
-    const uint32_t a2 = pack_bf16x2(x[2 * kk + 1][0], x[2 * kk + 1][1]);
-    const uint32_t a3 = pack_bf16x2(x[2 * kk + 1][2], x[2 * kk + 1][3]);
-#pragma unroll
-    for (int nd = 0; nd < D / 16; ++nd) {
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_trans(b_addr + (kk * 16 * RS + nd * 16) * 2, b0, b1, b2, b3);
-      mma_16816(out[2 * nd], a0, a1, a2, a3, b0, b1);
-      mma_16816(out[2 * nd + 1], a0, a1, a2, a3, b2, b3);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 128);
     }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
   }
-}
-
-template <int D>
-__device__ __forceinline__ void bwd_store(__nv_bfloat16* dst, const float (&acc)[D / 8][4], float mul, int64_t bh,
-                                          int N, int r0, int lane) {
-  const int g4 = lane >> 2, t4 = lane & 3;
-#pragma unroll
-  for (int n = 0; n < D / 8; ++n) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int r = r0 + g4 + 8 * h;
-      if (r < N)
-        *reinterpret_cast<uint32_t*>(dst + (bh * N + r) * D + n * 8 + 2 * t4) =
-            pack_bf16x2(acc[n][2 * h] * mul, acc[n][2 * h + 1] * mul);
-    }
+  if (warp == 5) {
+    tmem_alloc(tmem_base_s, C::kTmemCols);
+    tmem_relinquish();
   }
-}
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t taddr = *tmem_base_s;
 
-template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkv_kernel(BwdParams p) {
-  extern __shared__ __align__(16) __nv_bfloat16 bwd_smem[];
-  constexpr int RS = D + 8;
-  __nv_bfloat16* ks = bwd_smem;
-  __nv_bfloat16* vs = ks + kBwdTile * RS;
-  __nv_bfloat16* qs = vs + kBwdTile * RS;
-  __nv_bfloat16* dos = qs + kBwdTile * RS;
-  __shared__ float lse_s[kBwdTile], dot_s[kBwdTile];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g4 = lane >> 2, t4 = lane & 3;
-  const int64_t bh = blockIdx.y;
-  const int key0 = blockIdx.x * kBwdTile;
-  const int J = key0 / p.block;
-  const float c2 = p.scale * 1.4426950408889634f;
-  bwd_stage<D>(ks, p.k, bh, p.N, key0);
-  bwd_stage<D>(vs, p.v, bh, p.N, key0);
-  float acc_dk[D / 8][4], acc_dv[D / 8][4];
-#pragma unroll
-  for (int n = 0; n < D / 8; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc_dk[n][e] = acc_dv[n][e] = 0.f;
-  const int tiles_per_block = p.block / kBwdTile;
-  const int64_t tr = bh * p.nb + J;
-  for (int c = p.t_ptr[tr]; c < p.t_ptr[tr + 1]; ++c) {
-    const int I = p.t_col[c];
-    for (int qt = 0; qt < tiles_per_block; ++qt) {
-      const int q0 = I * p.block + qt * kBwdTile;
-      if (q0 >= p.N) break;
-      __syncthreads();   // the previous tile's Q / dO are consumed
-      bwd_stage<D>(qs, p.q, bh, p.N, q0);
-      bwd_stage<D>(dos, p.dout, bh, p.N, q0);
-      for (int r = threadIdx.x; r < kBwdTile; r += kBwdThreads) {
-        const bool in = q0 + r < p.N;
-        lse_s[r] = in ? p.lse[bh * p.N + q0 + r] * 1.4426950408889634f : INFINITY;   // padded rows: P = 0
-        dot_s[r] = in ? p.rowdot[bh * p.N + q0 + r] : 0.f;
+  if (warp == 4) {
+    // ------------------------------------------------------------- producer
+    int32_t ptr = 0, end = 0, cur = INT32_MAX;
+    if (lane < C::kR && blk0 + lane < nb) {
+      const int64_t r = static_cast<int64_t>(bh) * nb + blk0 + lane;
+      ptr = KV ? p.t_ptr[r] : p.row_ptr[r];
+      end = KV ? p.t_ptr[r + 1] : p.row_ptr[r + 1];
+      const int32_t* lst = KV ? p.t_col : p.col_idx;
+      while (ptr < end) {
+        const int32_t c = lst[ptr];
+        if (c >= 0 && c < nb) { cur = c; break; }
+        record_error(DYNRAD_ERR_DEVICE);
+        ++ptr;
       }
-      __syncthreads();
-      float s[8][4], dp[8][4];
+    }
+    if (lane == 0) {
+      prefetch_tensormap(&tm_res0);
+      prefetch_tensormap(&tm_res1);
+      prefetch_tensormap(&tm_step0);
+      prefetch_tensormap(&tm_step1);
+      mbar_arrive_expect_tx(res_full, 2 * C::kResBytes);
 #pragma unroll
-      for (int n = 0; n < 8; ++n)
+      for (int c = 0; c < C::kChunks; ++c) {
+        tma_load_3d(res_smem + c * C::kResChunk, &tm_res0, res_full, c * 64, tile0, bh);
+        tma_load_3d(res_smem + C::kResBytes + c * C::kResChunk, &tm_res1, res_full, c * 64, tile0, bh);
+      }
+    }
+    const int32_t* lst = KV ? p.t_col : p.col_idx;
+    bool ok = true;
+    int j = 0;   // steps published
+    auto slot_ready = [&](int i) -> bool {
+      bool w = true;
+      if (i >= NS && lane == 0) w = mbar_wait(&slot_empty[i % NS], ((i / NS) - 1) & 1, abort_flag);
+      return __shfl_sync(0xffffffffu, w, 0);
+    };
+    for (;;) {
+      int32_t m = cur;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) s[n][e] = dp[n][e] = 0.f;
-      bwd_rows_by_rows<D>(s, ks, qs, warp * 16, lane);    // S^T: keys x queries
-      bwd_rows_by_rows<D>(dp, vs, dos, warp * 16, lane);  // dP^T
-#pragma unroll
-      for (int n = 0; n < 8; ++n) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int key = key0 + warp * 16 + g4 + 8 * (e >> 1);
-          const int qi = n * 8 + 2 * t4 + (e & 1);
-          const float pv = key < p.N ? exp2f(s[n][e] * c2 - lse_s[qi]) : 0.f;
-          s[n][e] = pv;
-          dp[n][e] = pv * (dp[n][e] - dot_s[qi]);
+      for (int off = 16; off > 0; off >>= 1) m = min(m, __shfl_xor_sync(0xffffffffu, m, off));
+      const bool mine = lane < C::kR && cur == m && m != INT32_MAX;
+      const uint32_t mask = __ballot_sync(0xffffffffu, mine);
+      if (mine) {
+        ++ptr;
+        cur = INT32_MAX;
+        while (ptr < end) {
+          const int32_t c = lst[ptr];
+          if (c > m && c < nb) { cur = c; break; }
+          record_error(DYNRAD_ERR_DEVICE);
+          ++ptr;
         }
       }
-      bwd_acc_times_rows<D>(acc_dv, s, dos, lane);   // dV += P^T dO
-      bwd_acc_times_rows<D>(acc_dk, dp, qs, lane);   // dK += dS^T Q
+      if (m == INT32_MAX) {
+        // end marker: a slot with no tiles
+        if (!slot_ready(j)) { ok = false; break; }
+        if (lane == 0) {
+          BwdStepMeta* mt = reinterpret_cast<BwdStepMeta*>(slot_tail(j) + 512);
+          mt->row0 = 0;
+          mt->mask = 0u;
+          mt->end = 1;
+        }
+        __syncwarp();
+        mbar_arrive(&slot_full[j % NS]);
+        break;
+      }
+      for (int s = 0; s < C::kSPB; ++s) {
+        const int row0 = m * BS + s * C::kStep;
+        if (row0 >= p.N) break;
+        if (!slot_ready(j)) { ok = false; break; }
+        uint8_t* tail = slot_tail(j);
+        if (KV) {
+          float* lse2 = reinterpret_cast<float*>(tail);
+          float* dr = lse2 + 64;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int q = row0 + h * 32 + lane;
+            const bool in = q < p.N;
+            lse2[h * 32 + lane] = in ? p.lse[static_cast<int64_t>(bh) * p.N + q] * log2e : INFINITY;
+            dr[h * 32 + lane] = in ? p.rowdot[static_cast<int64_t>(bh) * p.N + q] : 0.f;
+          }
+        }
+        if (lane == 0) {
+          BwdStepMeta* mt = reinterpret_cast<BwdStepMeta*>(tail + 512);
+          mt->row0 = row0;
+          mt->mask = mask;
+          mt->end = 0;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&slot_full[j % NS], 2 * C::kStepBytes);
+#pragma unroll
+          for (int c = 0; c < C::kChunks; ++c) {
+            tma_load_3d(slot_tile(j, 0) + c * C::kStepChunk, &tm_step0, &slot_full[j % NS], c * 64, row0, bh);
+            tma_load_3d(slot_tile(j, 1) + c * C::kStepChunk, &tm_step1, &slot_full[j % NS], c * 64, row0, bh);
+          }
+        } else {
+          mbar_arrive(&slot_full[j % NS]);
+        }
+        ++j;
+      }
+      if (!ok) break;
     }
-  }
-  bwd_store<D>(p.dk, acc_dk, p.scale, bh, p.N, key0 + warp * 16, lane);
-  bwd_store<D>(p.dv, acc_dv, 1.0f, bh, p.N, key0 + warp * 16, lane);
-}
-
-template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(BwdParams p) {
-  extern __shared__ __align__(16) __nv_bfloat16 bwd_smem[];
-  constexpr int RS = D + 8;
-  __nv_bfloat16* qs = bwd_smem;
-  __nv_bfloat16* dos = qs + kBwdTile * RS;
-  __nv_bfloat16* ks = dos + kBwdTile * RS;
-  __nv_bfloat16* vs = ks + kBwdTile * RS;
-  __shared__ float lse_s[kBwdTile], dot_s[kBwdTile];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g4 = lane >> 2, t4 = lane & 3;
-  const int64_t bh = blockIdx.y;
-  const int q0 = blockIdx.x * kBwdTile;
-  const int I = q0 / p.block;
-  const float c2 = p.scale * 1.4426950408889634f;
-  bwd_stage<D>(qs, p.q, bh, p.N, q0);
-  bwd_stage<D>(dos, p.dout, bh, p.N, q0);
-  for (int r = threadIdx.x; r < kBwdTile; r += kBwdThreads) {
-    const bool in = q0 + r < p.N;
-    lse_s[r] = in ? p.lse[bh * p.N + q0 + r] * 1.4426950408889634f : INFINITY;
-    dot_s[r] = in ? p.rowdot[bh * p.N + q0 + r] : 0.f;
-  }
-  float acc_dq[D / 8][4];
+    if (!ok && lane == 0) {
+      for (int i = (j > NS ? j - NS : 0); i < j; ++i) mbar_wait(&slot_full[i % NS], (i / NS) & 1, nullptr);
+      mbar_wait(res_full, 0, nullptr);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc_g12 = idesc_bf16_f32(128, 64, false, false);
+      constexpr uint32_t idesc_g34 = idesc_bf16_f32(128, D, false, true);
+      const uint32_t res_base = smem_u32(res_smem);
+      bool ok = mbar_wait(res_full, 0, abort_flag);
+      bool started = false;
+      // G12 of step j into buffer j & 1; false at the end marker (or abort)
+      auto issue_g12 = [&](int j, bool& more) -> bool {
+        if (!mbar_wait(&slot_full[j % NS], (j / NS) & 1, abort_flag)) return false;
+        const BwdStepMeta* mt = reinterpret_cast<const BwdStepMeta*>(slot_tail(j) + 512);
+        more = mt->end == 0;
+        if (!more) return true;
+        tc_fence_after();
+        const int b = j & 1;
+        const uint32_t s0 = smem_u32(slot_tile(j, 0)), s1 = smem_u32(slot_tile(j, 1));
 #pragma unroll
-  for (int n = 0; n < D / 8; ++n)
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int c = kk >> 2, off = (kk & 3) * 32;
+          mma_ss(taddr + C::col_x(b), smem_desc_sw128(res_base + c * C::kResChunk + off, 16, 1024),
+                 smem_desc_sw128(s0 + c * C::kStepChunk + off, 16, 1024), idesc_g12, kk > 0 ? 1u : 0u);
+        }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc_dq[n][e] = 0.f;
-  const int tiles_per_block = p.block / kBwdTile;
-  const int64_t row = bh * p.nb + I;
-  for (int c = p.row_ptr[row]; c < p.row_ptr[row + 1]; ++c) {
-    const int J = p.col_idx[c];
-    if (J < 0 || J >= p.nb) continue;
-    for (int kt = 0; kt < tiles_per_block; ++kt) {
-      const int k0 = J * p.block + kt * kBwdTile;
-      if (k0 >= p.N) break;
-      __syncthreads();
-      bwd_stage<D>(ks, p.k, bh, p.N, k0);
-      bwd_stage<D>(vs, p.v, bh, p.N, k0);
-      __syncthreads();
-      float s[8][4], dp[8][4];
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int c = kk >> 2, off = (kk & 3) * 32;
+          mma_ss(taddr + C::col_y(b),
+                 smem_desc_sw128(res_base + C::kResBytes + c * C::kResChunk + off, 16, 1024),
+                 smem_desc_sw128(s1 + c * C::kStepChunk + off, 16, 1024), idesc_g12, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&s_full[b]);
+        return true;
+      };
+      bool more[2] = {false, false};   // step j & 1 has its G12 issued
+      if (ok) ok = issue_g12(0, more[0]);
+      if (ok && more[0]) ok = issue_g12(1, more[1]);
+      for (int j = 0; ok && more[j & 1]; ++j) {
+        const int b = j & 1;
+        if (!mbar_wait(&p_full[b], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t s0 = smem_u32(slot_tile(j, 0)), s1 = smem_u32(slot_tile(j, 1));
 #pragma unroll
-      for (int n = 0; n < 8; ++n)
+        for (int kk = 0; kk < C::kStep / 16; ++kk) {
+          // the step tile [64 rows][D] as the MN-major B operand: 64-column
+          // chunks kStepChunk bytes apart, 8-row groups 1024 bytes apart
+          const uint32_t acc = (started || kk > 0) ? 1u : 0u;
+          if (KV) {
+            mma_ts(taddr + C::kAcc0, taddr + C::col_x(b) + kk * 8,
+                   smem_desc_sw128(s1 + kk * 2048, C::kStepChunk, 1024), idesc_g34, acc);
+            mma_ts(taddr + C::kAcc1, taddr + C::col_y(b) + kk * 8,
+                   smem_desc_sw128(s0 + kk * 2048, C::kStepChunk, 1024), idesc_g34, acc);
+          } else {
+            mma_ts(taddr + C::kAcc0, taddr + C::col_y(b) + kk * 8,
+                   smem_desc_sw128(s0 + kk * 2048, C::kStepChunk, 1024), idesc_g34, acc);
+          }
+        }
+        started = true;
+        mma_commit(&slot_empty[j % NS]);
+        // G12(j + 2) into buffer b, after G34(j) in issue order; only while
+        // step j + 1 exists (else the walk is over and no slot j + 2 comes)
+        bool m2 = false;
+        if (more[b ^ 1] && !issue_g12(j + 2, m2)) { ok = false; break; }
+        more[b] = m2;
+      }
+      mma_commit(drain);
+      mbar_wait(drain, 0, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------- elementwise
+    const int t = threadIdx.x;                       // tile row = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int row = tile0 + t;
+    const bool row_in = row < p.N;
+    const int rbit = t / BS;
+    const float c2 = p.scale * log2e;
+    float my_lse2 = INFINITY, my_dr = 0.f;
+    if (!KV && row_in) {
+      my_lse2 = p.lse[static_cast<int64_t>(bh) * p.N + row] * log2e;
+      my_dr = p.rowdot[static_cast<int64_t>(bh) * p.N + row];
+    }
+    bool ok = true;
+    int j = 0;
+    for (;; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&slot_full[j % NS], (j / NS) & 1, abort_flag))) { ok = false; break; }
+      const uint8_t* tail = slot_tail(j);
+      const BwdStepMeta mt = *reinterpret_cast<const BwdStepMeta*>(tail + 512);
+      if (mt.end) break;
+      const int b = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag))) { ok = false; break; }
+      tc_fence_after();
+      const bool kept = row_in && ((mt.mask >> rbit) & 1u);
+      const float* lse2_s = reinterpret_cast<const float*>(tail);
+      const float* dr_s = lse2_s + 64;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) s[n][e] = dp[n][e] = 0.f;
-      bwd_rows_by_rows<D>(s, qs, ks, warp * 16, lane);    // S: queries x keys
-      bwd_rows_by_rows<D>(dp, dos, vs, warp * 16, lane);  // dP
+      for (int h = 0; h < 2; ++h) {
+        uint32_t xr[32], yr[32];
+        tmem_ld32(taddr + lane_base + C::col_x(b) + h * 32, xr);
+        tmem_ld32(taddr + lane_base + C::col_y(b) + h * 32, yr);
+        tmem_wait_ld();
+        uint32_t pk[16], dk[16];
 #pragma unroll
-      for (int n = 0; n < 8; ++n) {
+        for (int i = 0; i < 32; i += 2) {
+          float pv[2], dv[2];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int qi = warp * 16 + g4 + 8 * (e >> 1);
-          const int key = k0 + n * 8 + 2 * t4 + (e & 1);
-          const float pv = key < p.N ? exp2f(s[n][e] * c2 - lse_s[qi]) : 0.f;
-          dp[n][e] = pv * (dp[n][e] - dot_s[qi]);
+          for (int u = 0; u < 2; ++u) {
+            const int col = h * 32 + i + u;
+            float l2, dd;
+            bool valid = kept;
+            if (KV) {
+              l2 = lse2_s[col];
+              dd = dr_s[col];
+            } else {
+              l2 = my_lse2;
+              dd = my_dr;
+              valid = valid && (mt.row0 + col < p.N);
+            }
+            const float e = ex2_approx(fmaf(__uint_as_float(xr[i + u]), c2, -l2));
+            pv[u] = valid ? e : 0.f;
+            dv[u] = pv[u] * (__uint_as_float(yr[i + u]) - dd);
+          }
+          pk[i / 2] = pack_bf16x2(pv[0], pv[1]);
+          dk[i / 2] = pack_bf16x2(dv[0], dv[1]);
+        }
+        if (KV) tmem_st16(taddr + lane_base + C::col_x(b) + h * 16, pk);
+        tmem_st16(taddr + lane_base + C::col_y(b) + h * 16, dk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[b]);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(drain, 0, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      const bool have = j > 0;
+#pragma unroll
+      for (int a = 0; a < (KV ? 2 : 1); ++a) {
+        // KV: a = 0 dV (scale 1), a = 1 dK (scale); else dQ (scale)
+        const uint32_t col = a == 0 ? C::kAcc0 : C::kAcc1;
+        const float mul = (KV && a == 0) ? 1.0f : p.scale;
+        __nv_bfloat16* dst = KV ? (a == 0 ? p.dv : p.dk) : p.dq;
+        __nv_bfloat16* drow = dst + (static_cast<int64_t>(bh) * p.N + row) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          if (have) {
+            tmem_ld32(taddr + lane_base + col + c * 32, r);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = 0u;
+          }
+          uint32_t packed[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            packed[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * mul, __uint_as_float(r[2 * i + 1]) * mul);
+          if (row_in) {
+            uint4* d4 = reinterpret_cast<uint4*>(drow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              d4[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+          }
         }
       }
-      bwd_acc_times_rows<D>(acc_dq, dp, ks, lane);   // dQ += dS K
     }
   }
-  bwd_store<D>(p.dq, acc_dq, p.scale, bh, p.N, q0 + warp * 16, lane);
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(taddr, C::kTmemCols);
 }
 
 }  // namespace dynrad

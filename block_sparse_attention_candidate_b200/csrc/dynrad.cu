@@ -739,24 +739,34 @@ BwdWorkspace bwd_layout(int64_t bh, int64_t n, int64_t nb, int64_t col_cap) {
   return w;
 }
 
-template <int D>
-int launch_backward(const BwdParams& bp, cudaStream_t st) {
-  const size_t smem = static_cast<size_t>(4) * kBwdTile * (D + 8) * 2;
-  static bool attr = false;
+template <int D, int BS, bool KV>
+int launch_bwd_tc(const BwdParams& bp, const CUtensorMap& r0, const CUtensorMap& r1, const CUtensorMap& s0,
+                  const CUtensorMap& s1, cudaStream_t st) {
+  using C = BwdTcCfg<D, BS, KV>;
+  static bool attr = false;   // per instantiation
   if (!attr) {
-    if (cudaFuncSetAttribute(bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess ||
-        cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
+    if (cudaFuncSetAttribute(bwd_tc_kernel<D, BS, KV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemTotal) != cudaSuccess)
       return DYNRAD_ERR_CUDA;
     attr = true;
   }
-  const dim3 grid((bp.N + kBwdTile - 1) / kBwdTile, bp.BH);
-  bwd_dkv_kernel<D><<<grid, kBwdThreads, smem, st>>>(bp);
-  int rc = launch_status();
-  if (rc != DYNRAD_OK) return rc;
-  bwd_dq_kernel<D><<<grid, kBwdThreads, smem, st>>>(bp);
+  const dim3 grid((bp.N + C::kRows - 1) / C::kRows, bp.BH);
+  bwd_tc_kernel<D, BS, KV><<<grid, 192, C::kSmemTotal, st>>>(r0, r1, s0, s1, bp);
   return launch_status();
+}
+
+// dK / dV (resident K, V; streamed Q, dO), then dQ (resident Q, dO; streamed K, V)
+template <int D, int BS>
+int launch_backward(const BwdParams& bp, cudaStream_t st) {
+  CUtensorMap k128, v128, q64, do64, q128, do128, k64, v64;
+  if (!encode_map(&k128, bp.k, D, bp.N, bp.BH, 128) || !encode_map(&v128, bp.v, D, bp.N, bp.BH, 128) ||
+      !encode_map(&q64, bp.q, D, bp.N, bp.BH, 64) || !encode_map(&do64, bp.dout, D, bp.N, bp.BH, 64) ||
+      !encode_map(&q128, bp.q, D, bp.N, bp.BH, 128) || !encode_map(&do128, bp.dout, D, bp.N, bp.BH, 128) ||
+      !encode_map(&k64, bp.k, D, bp.N, bp.BH, 64) || !encode_map(&v64, bp.v, D, bp.N, bp.BH, 64))
+    return DYNRAD_ERR_CUDA;
+  const int rc = launch_bwd_tc<D, BS, true>(bp, k128, v128, q64, do64, st);
+  if (rc != DYNRAD_OK) return rc;
+  return launch_bwd_tc<D, BS, false>(bp, q128, do128, k64, v64, st);
 }
 
 }  // namespace
@@ -844,7 +854,8 @@ int dynrad_attn_backward(const void* q, const void* k, const void* v, const void
   }
   bwd_tfill_kernel<<<wblocks, 256, 0, st>>>(bp);
   if ((rc = launch_status()) != DYNRAD_OK) return rc;
-  return D == 128 ? launch_backward<128>(bp, st) : launch_backward<64>(bp, st);
+  if (D == 128) return block == 64 ? launch_backward<128, 64>(bp, st) : launch_backward<128, 128>(bp, st);
+  return block == 64 ? launch_backward<64, 64>(bp, st) : launch_backward<64, 128>(bp, st);
 }
 
 int dynrad_sparse_attn(const void* q, const void* k, const void* v, int32_t B, int32_t H, int32_t N,
