@@ -7,7 +7,8 @@
 //   dQ = scale dS K,  dK = scale dS^T Q.
 //
 // Kernels:
-//   bwd_rowdot_kernel     D_r per query row.
+//   bwd_aux_kernel        per query row the pair (lse log2(e), D_r), rows
+//                         padded to a multiple of 64 with (+inf, 0).
 //   bwd_tcount_kernel, scan, bwd_tfill_kernel   the transposed CSR: for each
 //                         key block, the query blocks that keep it, ascending.
 //   bwd_tc_kernel<D, BS, true>   dK, dV per 128-key tile (tcgen05, TMEM, TMA).
@@ -28,7 +29,8 @@ struct BwdParams {
   const __nv_bfloat16* o;
   const __nv_bfloat16* dout;
   const float* lse;         // [BH, N] natural log
-  float* rowdot;            // [BH, N] D_r
+  float2* aux;              // [BH, Np]: (lse * log2(e), D_r); rows >= N: (+inf, 0)
+  int Np;                   // N rounded up to 64
   const int32_t* row_ptr;   // [BH * nb + 1]
   const int32_t* col_idx;
   int32_t* t_ptr;           // [BH * nb + 1] transposed CSR
@@ -41,16 +43,23 @@ struct BwdParams {
   float scale;              // logit scale
 };
 
-__global__ void bwd_rowdot_kernel(BwdParams p, int D) {
-  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+__global__ void bwd_aux_kernel(BwdParams p, int D) {
+  const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (row >= static_cast<int64_t>(p.BH) * p.N) return;
+  if (r >= static_cast<int64_t>(p.BH) * p.Np) return;
+  const int64_t bh = r / p.Np;
+  const int i = static_cast<int>(r - bh * p.Np);
+  if (i >= p.N) {
+    if (lane == 0) p.aux[r] = make_float2(INFINITY, 0.f);
+    return;
+  }
+  const int64_t row = bh * p.N + i;
   float s = 0.f;
   for (int d = lane; d < D; d += 32)
     s = fmaf(__bfloat162float(p.dout[row * D + d]), __bfloat162float(p.o[row * D + d]), s);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) p.rowdot[row] = s;
+  if (lane == 0) p.aux[r] = make_float2(p.lse[row] * 1.4426950408889634f, s);
 }
 
 // one warp per (head, query block): count its key blocks
@@ -119,18 +128,19 @@ __global__ void bwd_tfill_kernel(BwdParams p) {
 //   G12  X_b = A0 B0^T, Y_b = A1 B1^T (A = resident tiles, B = the step's
 //        tiles; M = 128, N = 64, K = D).  KV: X = S^T, Y = dP^T; else X = S,
 //        Y = dP.
-//   elementwise (warps 0-3, thread = TMEM lane = tile row): P = 2^(X c - lse2),
-//        dS = P (Y - D_r); P (KV only) and dS are written back as bf16 pairs
-//        over the first 32 columns of X_b and Y_b.
+//   elementwise (warps 0-7; thread = TMEM lane = tile row, warpgroup g = the
+//        32-column half g of the step): P = 2^(X c - lse2), dS = P (Y - D_r);
+//        P (KV only) and dS are written back as bf16 pairs over the first 32
+//        columns of X_b and Y_b, once both warpgroups have read their halves.
 //   G34  KV: dV += P^T B1, dK += dS^T B0; else dQ += dS B0 (A from tensor
 //        memory, B = the step's tile as the MN-major operand; M = 128, N = D,
 //        K = 64).
 // The MMA thread issues G34(j) and then G12(j + 2) into the same buffer, so
 // the tensor core overlaps step j + 1's G12 with step j's elementwise work.
 //
-// Warp roles (192 threads): warps 0-3 elementwise and epilogue, warp 4
+// Warp roles (320 threads): warps 0-7 elementwise and epilogue, warp 8
 // producer (list walk, TMA loads into a ring of slots, per-query lse2 / D_r of
-// the step for KV), warp 5 MMA issuer.  Tensor memory (512 columns): acc0 at 0
+// the step for KV), warp 9 MMA issuer.  Tensor memory (512 columns): acc0 at 0
 // (dV or dQ), acc1 at D (dK), X_b at 2D' + 64 b, Y_b at 2D' + 128 + 64 b with
 // D' = D for KV and D / 2 otherwise.  Every wait is bounded (common.cuh).
 // ----------------------------------------------------------------------------
@@ -152,7 +162,8 @@ struct BwdTcCfg {
   static constexpr int kResChunk = kRows * 128;
   static constexpr int kStepBytes = kStep * D * 2;
   static constexpr int kStepChunk = kStep * 128;
-  static constexpr int kSlotBytes = 2 * kStepBytes + 1024;   // two tiles, lse2 / D_r / meta
+  static constexpr int kSlotBytes = 2 * kStepBytes + 1024;   // two tiles, (lse2, D_r) x 64, meta
+  static constexpr int kAuxBytes = KV ? 64 * 8 : 0;
   static constexpr int kSmemCtrl = 1024;
   static constexpr int kBudget = 227 * 1024 - kSmemCtrl - 1024;
   static constexpr int kSlotsRaw = (kBudget - 2 * kResBytes) / kSlotBytes;
@@ -173,10 +184,10 @@ struct BwdTcCfg {
 };
 
 template <int D, int BS, bool KV>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_res0, const __grid_constant__ CUtensorMap tm_res1,
                   const __grid_constant__ CUtensorMap tm_step0, const __grid_constant__ CUtensorMap tm_step1,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tm_aux, const BwdParams p) {
   using C = BwdTcCfg<D, BS, KV>;
   constexpr int NS = C::kSlots;
   extern __shared__ uint8_t bwd_smem_raw[];
@@ -192,7 +203,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* s_full = slot_empty + NS;     // [2]
   uint64_t* p_full = s_full + 2;          // [2]
   uint64_t* drain = p_full + 2;
-  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* rd_done = drain + 1;          // [2] both halves have read X_b, Y_b
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(rd_done + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_s + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -213,13 +225,14 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 128);
+      mbar_init(&p_full[b], 256);
+      mbar_init(&rd_done[b], 256);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_base_s, C::kTmemCols);
     tmem_relinquish();
   }
@@ -228,26 +241,30 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t taddr = *tmem_base_s;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------- producer
-    int32_t ptr = 0, end = 0, cur = INT32_MAX;
+    // lane r < R walks list r; `nxt` holds the entry after `cur`, loaded one
+    // union member ahead so the walk does not wait on memory
+    const int32_t* lst = KV ? p.t_col : p.col_idx;
+    int32_t ptr = 0, end = 0, cur = INT32_MAX, nxt = INT32_MAX;
     if (lane < C::kR && blk0 + lane < nb) {
       const int64_t r = static_cast<int64_t>(bh) * nb + blk0 + lane;
       ptr = KV ? p.t_ptr[r] : p.row_ptr[r];
       end = KV ? p.t_ptr[r + 1] : p.row_ptr[r + 1];
-      const int32_t* lst = KV ? p.t_col : p.col_idx;
       while (ptr < end) {
         const int32_t c = lst[ptr];
         if (c >= 0 && c < nb) { cur = c; break; }
         record_error(DYNRAD_ERR_DEVICE);
         ++ptr;
       }
+      if (ptr + 1 < end) nxt = lst[ptr + 1];
     }
     if (lane == 0) {
       prefetch_tensormap(&tm_res0);
       prefetch_tensormap(&tm_res1);
       prefetch_tensormap(&tm_step0);
       prefetch_tensormap(&tm_step1);
+      if (KV) prefetch_tensormap(&tm_aux);
       mbar_arrive_expect_tx(res_full, 2 * C::kResBytes);
 #pragma unroll
       for (int c = 0; c < C::kChunks; ++c) {
@@ -255,7 +272,6 @@ __global__ void __launch_bounds__(192, 1)
         tma_load_3d(res_smem + C::kResBytes + c * C::kResChunk, &tm_res1, res_full, c * 64, tile0, bh);
       }
     }
-    const int32_t* lst = KV ? p.t_col : p.col_idx;
     bool ok = true;
     int j = 0;   // steps published
     auto slot_ready = [&](int i) -> bool {
@@ -270,10 +286,12 @@ __global__ void __launch_bounds__(192, 1)
       const bool mine = lane < C::kR && cur == m && m != INT32_MAX;
       const uint32_t mask = __ballot_sync(0xffffffffu, mine);
       if (mine) {
+        // advance past m, skipping malformed entries (out of range or not ascending)
         ++ptr;
         cur = INT32_MAX;
         while (ptr < end) {
-          const int32_t c = lst[ptr];
+          const int32_t c = nxt;
+          nxt = ptr + 1 < end ? lst[ptr + 1] : INT32_MAX;
           if (c > m && c < nb) { cur = c; break; }
           record_error(DYNRAD_ERR_DEVICE);
           ++ptr;
@@ -297,31 +315,19 @@ __global__ void __launch_bounds__(192, 1)
         if (row0 >= p.N) break;
         if (!slot_ready(j)) { ok = false; break; }
         uint8_t* tail = slot_tail(j);
-        if (KV) {
-          float* lse2 = reinterpret_cast<float*>(tail);
-          float* dr = lse2 + 64;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int q = row0 + h * 32 + lane;
-            const bool in = q < p.N;
-            lse2[h * 32 + lane] = in ? p.lse[static_cast<int64_t>(bh) * p.N + q] * log2e : INFINITY;
-            dr[h * 32 + lane] = in ? p.rowdot[static_cast<int64_t>(bh) * p.N + q] : 0.f;
-          }
-        }
         if (lane == 0) {
           BwdStepMeta* mt = reinterpret_cast<BwdStepMeta*>(tail + 512);
           mt->row0 = row0;
           mt->mask = mask;
           mt->end = 0;
-        }
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&slot_full[j % NS], 2 * C::kStepBytes);
+          mbar_arrive_expect_tx(&slot_full[j % NS], 2 * C::kStepBytes + C::kAuxBytes);
 #pragma unroll
           for (int c = 0; c < C::kChunks; ++c) {
             tma_load_3d(slot_tile(j, 0) + c * C::kStepChunk, &tm_step0, &slot_full[j % NS], c * 64, row0, bh);
             tma_load_3d(slot_tile(j, 1) + c * C::kStepChunk, &tm_step1, &slot_full[j % NS], c * 64, row0, bh);
           }
+          // (lse2, D_r) of the step's 64 queries: 128 floats at x = 2 row0
+          if (KV) tma_load_2d(tail, &tm_aux, &slot_full[j % NS], 2 * row0, bh);
         } else {
           mbar_arrive(&slot_full[j % NS]);
         }
@@ -333,7 +339,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int i = (j > NS ? j - NS : 0); i < j; ++i) mbar_wait(&slot_full[i % NS], (i / NS) & 1, nullptr);
       mbar_wait(res_full, 0, nullptr);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA
     if (lane == 0) {
       constexpr uint32_t idesc_g12 = idesc_bf16_f32(128, 64, false, false);
@@ -403,16 +409,18 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------- elementwise
-    const int t = threadIdx.x;                       // tile row = TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int t = threadIdx.x & 127;                 // tile row = TMEM lane
+    const int g = warp >> 2;                         // column half of each step
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int row = tile0 + t;
     const bool row_in = row < p.N;
     const int rbit = t / BS;
     const float c2 = p.scale * log2e;
     float my_lse2 = INFINITY, my_dr = 0.f;
     if (!KV && row_in) {
-      my_lse2 = p.lse[static_cast<int64_t>(bh) * p.N + row] * log2e;
-      my_dr = p.rowdot[static_cast<int64_t>(bh) * p.N + row];
+      const float2 a = p.aux[static_cast<int64_t>(bh) * p.Np + row];
+      my_lse2 = a.x;
+      my_dr = a.y;
     }
     bool ok = true;
     int j = 0;
@@ -425,41 +433,53 @@ __global__ void __launch_bounds__(192, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
       const bool kept = row_in && ((mt.mask >> rbit) & 1u);
-      const float* lse2_s = reinterpret_cast<const float*>(tail);
-      const float* dr_s = lse2_s + 64;
+      uint32_t xr[32], yr[32];
+      tmem_ld32(taddr + lane_base + C::col_x(b) + g * 32, xr);
+      tmem_ld32(taddr + lane_base + C::col_y(b) + g * 32, yr);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&rd_done[b]);
+      // KV: per column pair the step's (lse2, D_r) for queries q, q + 1;
+      // padded queries carry lse2 = +inf, so P = 0 there.  dQ side: per-row
+      // constants, keys past N masked on the sequence's last step only.
+      const float4* aux_s = reinterpret_cast<const float4*>(tail) + g * 16;
+      const float2 cc = make_float2(c2, c2);
+      const bool tail_step = !KV && mt.row0 + 64 > p.N;
+      uint32_t pk[16], dk[16];
+      if (!kept) {   // warp-uniform (the warp's 32 rows share one block) but at the sequence end
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t xr[32], yr[32];
-        tmem_ld32(taddr + lane_base + C::col_x(b) + h * 32, xr);
-        tmem_ld32(taddr + lane_base + C::col_y(b) + h * 32, yr);
-        tmem_wait_ld();
-        uint32_t pk[16], dk[16];
+        for (int i = 0; i < 16; ++i) pk[i] = dk[i] = 0u;
+      } else {
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float pv[2], dv[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int col = h * 32 + i + u;
-            float l2, dd;
-            bool valid = kept;
-            if (KV) {
-              l2 = lse2_s[col];
-              dd = dr_s[col];
-            } else {
-              l2 = my_lse2;
-              dd = my_dr;
-              valid = valid && (mt.row0 + col < p.N);
-            }
-            const float e = ex2_approx(fmaf(__uint_as_float(xr[i + u]), c2, -l2));
-            pv[u] = valid ? e : 0.f;
-            dv[u] = pv[u] * (__uint_as_float(yr[i + u]) - dd);
+        for (int i2 = 0; i2 < 16; ++i2) {
+          const int i = 2 * i2;   // column within the half
+          float2 l2, dd;
+          if (KV) {
+            const float4 a = aux_s[i2];
+            l2 = make_float2(-a.x, -a.z);
+            dd = make_float2(-a.y, -a.w);
+          } else {
+            l2 = make_float2(-my_lse2, -my_lse2);
+            dd = make_float2(-my_dr, -my_dr);
           }
-          pk[i / 2] = pack_bf16x2(pv[0], pv[1]);
-          dk[i / 2] = pack_bf16x2(dv[0], dv[1]);
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(xr[i]), __uint_as_float(xr[i + 1])), cc, l2);
+          float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          if (tail_step) {
+            const int k = mt.row0 + g * 32 + i;
+            pv.x = k < p.N ? pv.x : 0.f;
+            pv.y = k + 1 < p.N ? pv.y : 0.f;
+          }
+          const float2 y = __fadd2_rn(make_float2(__uint_as_float(yr[i]), __uint_as_float(yr[i + 1])), dd);
+          const float2 ds = __fmul2_rn(pv, y);
+          pk[i2] = pack_bf16x2(pv.x, pv.y);
+          dk[i2] = pack_bf16x2(ds.x, ds.y);
         }
-        if (KV) tmem_st16(taddr + lane_base + C::col_x(b) + h * 16, pk);
-        tmem_st16(taddr + lane_base + C::col_y(b) + h * 16, dk);
       }
+      // both halves have read X_b / Y_b before either overwrites its first 32 columns
+      if (!__all_sync(0xffffffffu, mbar_wait(&rd_done[b], (j >> 1) & 1, abort_flag))) { ok = false; break; }
+      tc_fence_after();
+      if (KV) tmem_st16(taddr + lane_base + C::col_x(b) + g * 16, pk);
+      tmem_st16(taddr + lane_base + C::col_y(b) + g * 16, dk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[b]);
@@ -470,13 +490,14 @@ __global__ void __launch_bounds__(192, 1)
       const bool have = j > 0;
 #pragma unroll
       for (int a = 0; a < (KV ? 2 : 1); ++a) {
-        // KV: a = 0 dV (scale 1), a = 1 dK (scale); else dQ (scale)
+        // KV: a = 0 dV (scale 1), a = 1 dK (scale); else dQ (scale).  Warpgroup
+        // g writes columns [g D / 2, (g + 1) D / 2).
         const uint32_t col = a == 0 ? C::kAcc0 : C::kAcc1;
         const float mul = (KV && a == 0) ? 1.0f : p.scale;
         __nv_bfloat16* dst = KV ? (a == 0 ? p.dv : p.dk) : p.dq;
         __nv_bfloat16* drow = dst + (static_cast<int64_t>(bh) * p.N + row) * D;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = g * (D / 64); c < (g + 1) * (D / 64); ++c) {
           uint32_t r[32];
           if (have) {
             tmem_ld32(taddr + lane_base + col + c * 32, r);
@@ -503,7 +524,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(taddr, C::kTmemCols);
+  if (warp == 9) tmem_dealloc(taddr, C::kTmemCols);
 }
 
 }  // namespace dynrad

@@ -126,6 +126,20 @@ bool encode_map(CUtensorMap* map, const void* base, int D, int N, int BH, int bo
   return r == CUDA_SUCCESS;
 }
 
+// 2-D map over the [BH, Np] float pairs of the backward: box = 64 pairs (512 B) x 1.
+bool encode_aux_map(CUtensorMap* map, const void* base, int Np, int BH) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(Np) * 2, static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(Np) * 8};
+  cuuint32_t box[2] = {128, 1};
+  cuuint32_t es[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int D, int BS>
 int launch_attn(const void* q, const void* k, const void* v, int BH, int N, const int32_t* row_ptr,
                 const int32_t* col_idx, float scale, void* o, float* lse, cudaStream_t st) {
@@ -724,15 +738,16 @@ int dynrad_build_token_mask(const void* q, const void* k, int32_t B, int32_t H, 
 namespace {
 
 struct BwdWorkspace {
-  size_t rowdot, t_ptr, t_col, partial, total;
+  size_t aux, t_ptr, t_col, partial, total;
 };
 
 BwdWorkspace bwd_layout(int64_t bh, int64_t n, int64_t nb, int64_t col_cap) {
   BwdWorkspace w;
   const int64_t rows = bh * nb;
   const int64_t tiles = (rows + 1 + kScanTile - 1) / kScanTile;
-  w.rowdot = 0;
-  w.t_ptr = align256(w.rowdot + static_cast<size_t>(bh * n) * 4);
+  const int64_t np = (n + 63) / 64 * 64;
+  w.aux = 0;
+  w.t_ptr = align256(w.aux + static_cast<size_t>(bh * np) * 8);
   w.t_col = align256(w.t_ptr + static_cast<size_t>(rows + 1) * 4);
   w.partial = align256(w.t_col + static_cast<size_t>(col_cap) * 4);
   w.total = align256(w.partial + static_cast<size_t>(tiles) * 8);
@@ -741,7 +756,7 @@ BwdWorkspace bwd_layout(int64_t bh, int64_t n, int64_t nb, int64_t col_cap) {
 
 template <int D, int BS, bool KV>
 int launch_bwd_tc(const BwdParams& bp, const CUtensorMap& r0, const CUtensorMap& r1, const CUtensorMap& s0,
-                  const CUtensorMap& s1, cudaStream_t st) {
+                  const CUtensorMap& s1, const CUtensorMap& aux, cudaStream_t st) {
   using C = BwdTcCfg<D, BS, KV>;
   static bool attr = false;   // per instantiation
   if (!attr) {
@@ -751,22 +766,23 @@ int launch_bwd_tc(const BwdParams& bp, const CUtensorMap& r0, const CUtensorMap&
     attr = true;
   }
   const dim3 grid((bp.N + C::kRows - 1) / C::kRows, bp.BH);
-  bwd_tc_kernel<D, BS, KV><<<grid, 192, C::kSmemTotal, st>>>(r0, r1, s0, s1, bp);
+  bwd_tc_kernel<D, BS, KV><<<grid, 320, C::kSmemTotal, st>>>(r0, r1, s0, s1, aux, bp);
   return launch_status();
 }
 
 // dK / dV (resident K, V; streamed Q, dO), then dQ (resident Q, dO; streamed K, V)
 template <int D, int BS>
 int launch_backward(const BwdParams& bp, cudaStream_t st) {
-  CUtensorMap k128, v128, q64, do64, q128, do128, k64, v64;
+  CUtensorMap k128, v128, q64, do64, q128, do128, k64, v64, aux;
   if (!encode_map(&k128, bp.k, D, bp.N, bp.BH, 128) || !encode_map(&v128, bp.v, D, bp.N, bp.BH, 128) ||
       !encode_map(&q64, bp.q, D, bp.N, bp.BH, 64) || !encode_map(&do64, bp.dout, D, bp.N, bp.BH, 64) ||
       !encode_map(&q128, bp.q, D, bp.N, bp.BH, 128) || !encode_map(&do128, bp.dout, D, bp.N, bp.BH, 128) ||
-      !encode_map(&k64, bp.k, D, bp.N, bp.BH, 64) || !encode_map(&v64, bp.v, D, bp.N, bp.BH, 64))
+      !encode_map(&k64, bp.k, D, bp.N, bp.BH, 64) || !encode_map(&v64, bp.v, D, bp.N, bp.BH, 64) ||
+      !encode_aux_map(&aux, bp.aux, bp.Np, bp.BH))
     return DYNRAD_ERR_CUDA;
-  const int rc = launch_bwd_tc<D, BS, true>(bp, k128, v128, q64, do64, st);
+  const int rc = launch_bwd_tc<D, BS, true>(bp, k128, v128, q64, do64, aux, st);
   if (rc != DYNRAD_OK) return rc;
-  return launch_bwd_tc<D, BS, false>(bp, q128, do128, k64, v64, st);
+  return launch_bwd_tc<D, BS, false>(bp, q128, do128, k64, v64, aux, st);
 }
 
 }  // namespace
@@ -810,7 +826,8 @@ int dynrad_attn_backward(const void* q, const void* k, const void* v, const void
   bp.o = static_cast<const __nv_bfloat16*>(o);
   bp.dout = static_cast<const __nv_bfloat16*>(dout);
   bp.lse = lse;
-  bp.rowdot = reinterpret_cast<float*>(ws + w.rowdot);
+  bp.aux = reinterpret_cast<float2*>(ws + w.aux);
+  bp.Np = (N + 63) / 64 * 64;
   bp.row_ptr = row_ptr;
   bp.col_idx = col_idx;
   bp.t_ptr = reinterpret_cast<int32_t*>(ws + w.t_ptr);
@@ -826,9 +843,9 @@ int dynrad_attn_backward(const void* q, const void* k, const void* v, const void
   bp.scale = scale == 0.0f ? 1.0f / std::sqrt(static_cast<float>(D)) : scale;
   int rc;
   const int64_t rows = bh * nb;
-  // D_r, then the transposed CSR
-  const int64_t nrows = bh * N;
-  bwd_rowdot_kernel<<<static_cast<unsigned>((nrows * 32 + 255) / 256), 256, 0, st>>>(bp, D);
+  // (lse2, D_r) per query row, then the transposed CSR
+  const int64_t nrows = bh * bp.Np;
+  bwd_aux_kernel<<<static_cast<unsigned>((nrows * 32 + 255) / 256), 256, 0, st>>>(bp, D);
   if ((rc = launch_status()) != DYNRAD_OK) return rc;
   if (cudaMemsetAsync(bp.t_ptr, 0, static_cast<size_t>(rows + 1) * 4, st) != cudaSuccess) return DYNRAD_ERR_CUDA;
   const unsigned wblocks = static_cast<unsigned>((rows * 32 + 255) / 256);

@@ -287,7 +287,8 @@ def test_backward_workspace_size_formula():
     rows = B * H * nb
     tiles = -(-(rows + 1) // 2048)
     got = L.dynrad_attn_backward_workspace_bytes(B, H, N, block, cap)
-    # D_r per query row (fp32), transposed CSR offsets and entries (int32), scan partials
-    need = B * H * N * 4 + (rows + 1) * 4 + cap * 4 + tiles * 8
+    # (lse log2 e, D_r) per query row padded to 64 rows (2 x fp32), transposed CSR
+    # offsets and entries (int32), scan partials
+    need = B * H * (-(-N // 64) * 64) * 8 + (rows + 1) * 4 + cap * 4 + tiles * 8
     assert need <= got < need + 4 * 256
     assert L.dynrad_attn_backward_workspace_bytes(0, H, N, block, cap) == 0
