@@ -69,6 +69,24 @@ def kept_flops(row_ptr: np.ndarray, col: np.ndarray, n: int, block: int, bh: int
     return float(4.0 * d * np.sum(rows_n.astype(np.float64) * kept_tok))
 
 
+def backward_tile_fill(row_ptr: np.ndarray, col: np.ndarray, bh: int, nb: int, block: int):
+    """Share of the backward's tensor-core tile area that kept pairs fill, per
+    side: a 128-row tile (128 / block blocks) streams the union of its blocks'
+    lists in 64-row steps, and a step's rows whose block lacks the member are
+    masked.  (dQ side: tiles of query blocks over their kept lists; dK/dV side:
+    tiles of key blocks over the query blocks that keep them.)"""
+    r = 128 // block
+    rows = np.repeat(np.arange(bh * nb, dtype=np.int64), np.diff(row_ptr[: bh * nb + 1]))
+    head, qb = rows // nb, rows % nb
+    useful = float(len(col))
+    out = {}
+    for side, tile_blk, member in (("dq", qb, col), ("dkv", col, qb)):
+        key = (head * nb + tile_blk // r) * nb + member
+        steps = len(np.unique(key)) * (block // 64)
+        out[side] = round(useful * block * block / (steps * 128.0 * 64.0), 4)
+    return out
+
+
 def max_over_ranks(x: float, device=None) -> float:
     """Max of a per-rank timing over all ranks (identity without a process group)."""
     import torch
@@ -537,8 +555,11 @@ def main():
         bwd_ms = e0.elapsed_time(e1) / reps
         # algorithmic backward FLOPs: S, dP, dV, dQ, dK products, 2.5x the forward's
         bflops = 2.5 * flops_run[0]
+        rpn = rp0.cpu().numpy().astype(np.int64)
+        coln = col0[: int(rpn[-1])].cpu().numpy().astype(np.int64)
         backward = {"run": r0["label"], "ms": round(bwd_ms, 3), "tflops": round(bflops / (bwd_ms * 1e-3) / 1e12, 1),
-                    "fwd_attn_ms": run_info[r0["label"]]["attn_ms"], "flop_model": "10 * D per kept (query, key)"}
+                    "fwd_attn_ms": run_info[r0["label"]]["attn_ms"], "flop_model": "10 * D per kept (query, key)",
+                    "tile_fill": backward_tile_fill(rpn, coln, B * H, r0["geom"].n_blocks, r0["geom"].block)}
         del dout, grads, bws
 
     # ---- end to end through the host-memory entry point: pinned host Q, K, V

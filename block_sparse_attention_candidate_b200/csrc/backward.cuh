@@ -7,8 +7,11 @@
 //   dQ = scale dS K,  dK = scale dS^T Q.
 //
 // Kernels:
-//   bwd_aux_kernel        per query row the pair (lse log2(e), D_r), rows
-//                         padded to a multiple of 64 with (+inf, 0).
+//   bwd_aux_kernel        per query row -lse log2(e) and -D_r, stored per pair of
+//                         rows (q even) as {-lse2_q, -lse2_q+1, -D_q, -D_q+1} so
+//                         the elementwise pass feeds them straight to paired
+//                         FP32 ops; rows padded to a multiple of 64 with
+//                         (-inf, 0).
 //   bwd_tcount_kernel, scan, bwd_tfill_kernel   the transposed CSR: for each
 //                         key block, the query blocks that keep it, ascending.
 //   bwd_tc_kernel<D, BS, true>   dK, dV per 128-key tile (tcgen05, TMEM, TMA).
@@ -29,7 +32,7 @@ struct BwdParams {
   const __nv_bfloat16* o;
   const __nv_bfloat16* dout;
   const float* lse;         // [BH, N] natural log
-  float2* aux;              // [BH, Np]: (lse * log2(e), D_r); rows >= N: (+inf, 0)
+  float* aux;               // [BH, Np / 2] x {-lse2 (2 rows), -D_r (2 rows)}; rows >= N: (-inf, 0)
   int Np;                   // N rounded up to 64
   const int32_t* row_ptr;   // [BH * nb + 1]
   const int32_t* col_idx;
@@ -43,14 +46,23 @@ struct BwdParams {
   float scale;              // logit scale
 };
 
+// Position of row i's -lse2 in the pair layout (its -D_r is 2 floats later).
+__host__ __device__ __forceinline__ int64_t bwd_aux_index(int64_t bh, int64_t np, int64_t i) {
+  return (bh * np + (i & ~static_cast<int64_t>(1))) * 2 + (i & 1);
+}
+
 __global__ void bwd_aux_kernel(BwdParams p, int D) {
   const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= static_cast<int64_t>(p.BH) * p.Np) return;
   const int64_t bh = r / p.Np;
   const int i = static_cast<int>(r - bh * p.Np);
+  float* dst = p.aux + bwd_aux_index(bh, p.Np, i);
   if (i >= p.N) {
-    if (lane == 0) p.aux[r] = make_float2(INFINITY, 0.f);
+    if (lane == 0) {
+      dst[0] = -INFINITY;
+      dst[2] = 0.f;
+    }
     return;
   }
   const int64_t row = bh * p.N + i;
@@ -59,7 +71,10 @@ __global__ void bwd_aux_kernel(BwdParams p, int D) {
     s = fmaf(__bfloat162float(p.dout[row * D + d]), __bfloat162float(p.o[row * D + d]), s);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) p.aux[r] = make_float2(p.lse[row] * 1.4426950408889634f, s);
+  if (lane == 0) {
+    dst[0] = -p.lse[row] * 1.4426950408889634f;
+    dst[2] = -s;
+  }
 }
 
 // one warp per (head, query block): count its key blocks
@@ -416,11 +431,11 @@ __global__ void __launch_bounds__(320, 1)
     const bool row_in = row < p.N;
     const int rbit = t / BS;
     const float c2 = p.scale * log2e;
-    float my_lse2 = INFINITY, my_dr = 0.f;
+    float my_nl2 = -INFINITY, my_ndr = 0.f;   // -lse2, -D_r of this row (dQ side)
     if (!KV && row_in) {
-      const float2 a = p.aux[static_cast<int64_t>(bh) * p.Np + row];
-      my_lse2 = a.x;
-      my_dr = a.y;
+      const float* a = p.aux + bwd_aux_index(bh, p.Np, row);
+      my_nl2 = a[0];
+      my_ndr = a[2];
     }
     bool ok = true;
     int j = 0;
@@ -439,8 +454,8 @@ __global__ void __launch_bounds__(320, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&rd_done[b]);
-      // KV: per column pair the step's (lse2, D_r) for queries q, q + 1;
-      // padded queries carry lse2 = +inf, so P = 0 there.  dQ side: per-row
+      // KV: per column pair q, q + 1 the step's {-lse2, -lse2, -D_r, -D_r};
+      // padded queries carry -lse2 = -inf, so P = 0 there.  dQ side: per-row
       // constants, keys past N masked on the sequence's last step only.
       const float4* aux_s = reinterpret_cast<const float4*>(tail) + g * 16;
       const float2 cc = make_float2(c2, c2);
@@ -456,11 +471,11 @@ __global__ void __launch_bounds__(320, 1)
           float2 l2, dd;
           if (KV) {
             const float4 a = aux_s[i2];
-            l2 = make_float2(-a.x, -a.z);
-            dd = make_float2(-a.y, -a.w);
+            l2 = make_float2(a.x, a.y);
+            dd = make_float2(a.z, a.w);
           } else {
-            l2 = make_float2(-my_lse2, -my_lse2);
-            dd = make_float2(-my_dr, -my_dr);
+            l2 = make_float2(my_nl2, my_nl2);
+            dd = make_float2(my_ndr, my_ndr);
           }
           const float2 x = __ffma2_rn(make_float2(__uint_as_float(xr[i]), __uint_as_float(xr[i + 1])), cc, l2);
           float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));

@@ -126,7 +126,8 @@ bool encode_map(CUtensorMap* map, const void* base, int D, int N, int BH, int bo
   return r == CUDA_SUCCESS;
 }
 
-// 2-D map over the [BH, Np] float pairs of the backward: box = 64 pairs (512 B) x 1.
+// 2-D map over the backward's per-row (-lse2, -D_r) array, [BH] x [2 Np] floats:
+// box = 128 floats (64 rows, 512 B) x 1.
 bool encode_aux_map(CUtensorMap* map, const void* base, int Np, int BH) {
   auto enc = tensor_map_encoder();
   if (enc == nullptr) return false;
@@ -826,7 +827,7 @@ int dynrad_attn_backward(const void* q, const void* k, const void* v, const void
   bp.o = static_cast<const __nv_bfloat16*>(o);
   bp.dout = static_cast<const __nv_bfloat16*>(dout);
   bp.lse = lse;
-  bp.aux = reinterpret_cast<float2*>(ws + w.aux);
+  bp.aux = reinterpret_cast<float*>(ws + w.aux);
   bp.Np = (N + 63) / 64 * 64;
   bp.row_ptr = row_ptr;
   bp.col_idx = col_idx;
