@@ -159,6 +159,16 @@ __global__ void bwd_tfill_kernel(BwdParams p) {
 // (dV or dQ), acc1 at D (dK), X_b at 2D' + 64 b, Y_b at 2D' + 128 + 64 b with
 // D' = D for KV and D / 2 otherwise.  Every wait is bounded (common.cuh).
 // ----------------------------------------------------------------------------
+// 2-D tiled TMA load (non-multicast) of the per-row (-lse2, -D_r) pairs.
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t c0, int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
 struct BwdStepMeta {
   int32_t row0;     // first streamed row of the step
   uint32_t mask;    // bit r: list r holds the union member
