@@ -7,14 +7,15 @@ ctypes with the same names:
 * ``dynrad_select_blocks``    -- pooled block scores, static-ratio or
   dynamic-threshold selection into CSR (Sec. 3.2);
 * ``dynrad_sparse_attn``      -- block-sparse attention forward, O and LSE
-  (Sec. 3.3, Eq. 13).
+  (Sec. 3.3, Eq. 13); ``dynrad_attn_backward`` is its gradient under the
+  same mask.
 
 ``workloads`` holds the seeded synthetic inputs.  The binding is imported
 lazily so that the workload generator can be used without a GPU.
 """
 
 _ABI_NAMES = ("dynrad_num_blocks", "dynrad_build_candidates", "dynrad_build_candidates_into", "dynrad_select_blocks",
-              "dynrad_sparse_attn", "dynrad_device_status", "dynrad_select_workspace_bytes",
+              "dynrad_sparse_attn", "dynrad_attn_backward", "dynrad_device_status", "dynrad_select_workspace_bytes",
               "SelectBuffers", "DynradError", "make_geom", "lib")
 
 
