@@ -400,9 +400,11 @@ int dynrad_proxy_error(const float *lse_dense, const float *lse_kept,
  *   dS_qk = P_qk (dO_q . v_k - D_q)
  *   dQ_q  = scale * sum_k dS_qk k_k,   dK_k = scale * sum_q dS_qk q_q
  * (the exact gradient of the forward's output; keys of unkept blocks get
- * dK = dV = 0, rows with no kept block get dQ = 0).  Warp-level bf16 tensor
- * core products with fp32 accumulation; no atomics (one CTA owns each 64-row
- * tile of dK/dV and of dQ).  The workspace holds D_q and the transposed CSR.
+ * dK = dV = 0, rows with no kept block get dQ = 0).  Tensor cores (tcgen05,
+ * bf16 operands -- P and dS are rounded to bf16 -- fp32 accumulation in
+ * TMEM); no atomics, deterministic: one CTA owns each 128-row tile of dK/dV
+ * and of dQ, so S and dP are computed twice (once per side).  The workspace
+ * holds -lse log2(e) and -D_q per query row and the transposed CSR.
  *
  *   q, k, v, o, dout  device bf16 [B, H, N, D], D = 64 or 128
  *   lse           device fp32 [B, H, N] (the forward's, natural log)
