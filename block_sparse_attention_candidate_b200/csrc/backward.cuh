@@ -139,7 +139,8 @@ __global__ void bwd_tfill_kernel(BwdParams p) {
 // mask bit r says whether list r holds the member: the tile rows of block r
 // get P = 0 otherwise.
 //
-// Per step j (buffer b = j & 1):
+// Per step j (buffer b = j mod NB; NB = 3 X / Y buffers where tensor memory
+// has room, 2 for dK / dV at D = 128):
 //   G12  X_b = A0 B0^T, Y_b = A1 B1^T (A = resident tiles, B = the step's
 //        tiles; M = 128, N = 64, K = D).  KV: X = S^T, Y = dP^T; else X = S,
 //        Y = dP.
@@ -150,14 +151,16 @@ __global__ void bwd_tfill_kernel(BwdParams p) {
 //   G34  KV: dV += P^T B1, dK += dS^T B0; else dQ += dS B0 (A from tensor
 //        memory, B = the step's tile as the MN-major operand; M = 128, N = D,
 //        K = 64).
-// The MMA thread issues G34(j) and then G12(j + 2) into the same buffer, so
-// the tensor core overlaps step j + 1's G12 with step j's elementwise work.
+// The MMA thread issues G34(j) and then G12(j + NB) into the same buffer, so
+// the tensor core runs the G12 of the next NB - 1 steps while step j's
+// elementwise pass runs.
 //
 // Warp roles (320 threads): warps 0-7 elementwise and epilogue, warp 8
 // producer (list walk, TMA loads into a ring of slots, per-query lse2 / D_r of
 // the step for KV), warp 9 MMA issuer.  Tensor memory (512 columns): acc0 at 0
-// (dV or dQ), acc1 at D (dK), X_b at 2D' + 64 b, Y_b at 2D' + 128 + 64 b with
-// D' = D for KV and D / 2 otherwise.  Every wait is bounded (common.cuh).
+// (dV or dQ), acc1 at D (dK, KV only), then X_b at base + 128 b and Y_b at
+// base + 128 b + 64 (base = 2D for KV, D otherwise).  Every wait is bounded
+// (common.cuh).
 // ----------------------------------------------------------------------------
 // 2-D tiled TMA load (non-multicast) of the per-row (-lse2, -D_r) pairs.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
@@ -199,12 +202,15 @@ struct BwdTcCfg {
   static constexpr uint32_t kAcc0 = 0;
   static constexpr uint32_t kAcc1 = D;
   static constexpr uint32_t kXY = KV ? 2 * D : D;
-  __host__ __device__ static constexpr uint32_t col_x(int b) { return kXY + 64u * b; }
-  __host__ __device__ static constexpr uint32_t col_y(int b) { return kXY + 128u + 64u * b; }
+  // X / Y buffers: as many 128-column pairs as tensor memory holds, at most 3
+  static constexpr int kBufs = (kTmemCols - kXY) / 128 > 3 ? 3 : static_cast<int>((kTmemCols - kXY) / 128);
+  __host__ __device__ static constexpr uint32_t col_x(int b) { return kXY + 128u * b; }
+  __host__ __device__ static constexpr uint32_t col_y(int b) { return kXY + 128u * b + 64u; }
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(BS == 64 || BS == 128, "block size");
-  static_assert(kSlots >= 3, "the MMA issue order needs three slots");
-  static_assert(kXY + 256 <= kTmemCols, "tensor memory");
+  static_assert(kBufs >= 2 && kXY + 128u * kBufs <= kTmemCols, "tensor memory");
+  // G12(j + kBufs) waits for step j + kBufs's slot, which is freed by G34(j + kBufs - kSlots)
+  static_assert(kSlots >= kBufs + 1, "slots for the MMA issue order");
   static_assert(kSmemTotal <= 227 * 1024, "shared memory");
 };
 
@@ -215,6 +221,7 @@ __global__ void __launch_bounds__(320, 1)
                   const __grid_constant__ CUtensorMap tm_aux, const BwdParams p) {
   using C = BwdTcCfg<D, BS, KV>;
   constexpr int NS = C::kSlots;
+  constexpr int NB = C::kBufs;
   extern __shared__ uint8_t bwd_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(bwd_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -225,11 +232,11 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* res_full = bar;
   uint64_t* slot_full = bar + 1;          // [NS]
   uint64_t* slot_empty = slot_full + NS;  // [NS]
-  uint64_t* s_full = slot_empty + NS;     // [2]
-  uint64_t* p_full = s_full + 2;          // [2]
-  uint64_t* drain = p_full + 2;
-  uint64_t* rd_done = drain + 1;          // [2] both halves have read X_b, Y_b
-  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(rd_done + 2);
+  uint64_t* s_full = slot_empty + NS;     // [NB]
+  uint64_t* p_full = s_full + NB;         // [NB]
+  uint64_t* drain = p_full + NB;
+  uint64_t* rd_done = drain + 1;          // [NB] both halves have read X_b, Y_b
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(rd_done + NB);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_s + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -248,7 +255,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&slot_full[s], 32);
       mbar_init(&slot_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NB; ++b) {
       mbar_init(&s_full[b], 1);
       mbar_init(&p_full[b], 256);
       mbar_init(&rd_done[b], 256);
@@ -372,14 +379,14 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t res_base = smem_u32(res_smem);
       bool ok = mbar_wait(res_full, 0, abort_flag);
       bool started = false;
-      // G12 of step j into buffer j & 1; false at the end marker (or abort)
+      // G12 of step j into buffer j % NB; false on abort, more = false at the end marker
       auto issue_g12 = [&](int j, bool& more) -> bool {
         if (!mbar_wait(&slot_full[j % NS], (j / NS) & 1, abort_flag)) return false;
         const BwdStepMeta* mt = reinterpret_cast<const BwdStepMeta*>(slot_tail(j) + 512);
         more = mt->end == 0;
         if (!more) return true;
         tc_fence_after();
-        const int b = j & 1;
+        const int b = j % NB;
         const uint32_t s0 = smem_u32(slot_tile(j, 0)), s1 = smem_u32(slot_tile(j, 1));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -397,12 +404,17 @@ __global__ void __launch_bounds__(320, 1)
         mma_commit(&s_full[b]);
         return true;
       };
-      bool more[2] = {false, false};   // step j & 1 has its G12 issued
-      if (ok) ok = issue_g12(0, more[0]);
-      if (ok && more[0]) ok = issue_g12(1, more[1]);
-      for (int j = 0; ok && more[j & 1]; ++j) {
-        const int b = j & 1;
-        if (!mbar_wait(&p_full[b], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+      int issued = 0;       // steps whose G12 has been issued
+      bool ended = false;   // the end marker has been read
+      for (int i = 0; ok && i < NB && !ended; ++i) {
+        bool more = false;
+        if (!issue_g12(i, more)) ok = false;
+        else if (more) ++issued;
+        else ended = true;
+      }
+      for (int j = 0; ok && j < issued; ++j) {
+        const int b = j % NB;
+        if (!mbar_wait(&p_full[b], (j / NB) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t s0 = smem_u32(slot_tile(j, 0)), s1 = smem_u32(slot_tile(j, 1));
 #pragma unroll
@@ -422,11 +434,14 @@ __global__ void __launch_bounds__(320, 1)
         }
         started = true;
         mma_commit(&slot_empty[j % NS]);
-        // G12(j + 2) into buffer b, after G34(j) in issue order; only while
-        // step j + 1 exists (else the walk is over and no slot j + 2 comes)
-        bool m2 = false;
-        if (more[b ^ 1] && !issue_g12(j + 2, m2)) { ok = false; break; }
-        more[b] = m2;
+        // G12(j + NB) into buffer b, after G34(j) in issue order; only while
+        // every step before it exists (else no slot j + NB comes)
+        if (!ended) {
+          bool more = false;
+          if (!issue_g12(j + NB, more)) { ok = false; break; }
+          if (more) ++issued;
+          else ended = true;
+        }
       }
       mma_commit(drain);
       mbar_wait(drain, 0, nullptr);
@@ -454,8 +469,8 @@ __global__ void __launch_bounds__(320, 1)
       const uint8_t* tail = slot_tail(j);
       const BwdStepMeta mt = *reinterpret_cast<const BwdStepMeta*>(tail + 512);
       if (mt.end) break;
-      const int b = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag))) { ok = false; break; }
+      const int b = j % NB;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (j / NB) & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
       const bool kept = row_in && ((mt.mask >> rbit) & 1u);
       uint32_t xr[32], yr[32];
@@ -501,7 +516,7 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       // both halves have read X_b / Y_b before either overwrites its first 32 columns
-      if (!__all_sync(0xffffffffu, mbar_wait(&rd_done[b], (j >> 1) & 1, abort_flag))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&rd_done[b], (j / NB) & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
       if (KV) tmem_st16(taddr + lane_base + C::col_x(b) + g * 16, pk);
       tmem_st16(taddr + lane_base + C::col_y(b) + g * 16, dk);
