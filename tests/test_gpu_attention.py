@@ -152,3 +152,17 @@ def test_fma_pipe_exp2_against_cuda_exp2f():
     low = torch.tensor([-1000.0, -200.0, -126.0], device="cuda")
     pl, _ = abi.dynrad_debug_exp2(low)
     assert bool(torch.isfinite(pl).all()) and float(pl.max()) < 1e-37
+
+
+@pytest.mark.parametrize("n", [1, 40, 100])
+@pytest.mark.parametrize("D,block", [(64, 32), (128, 64), (64, 128)])
+def test_sequences_shorter_than_one_tile(n, D, block):
+    # fewer tokens than one 128-row query tile (and than one block for n < block):
+    # the tensor maps' boxes run past the sequence and read zeros there
+    B, H = 1, 2
+    nb = -(-n // block)
+    bits = random_qkv_bf16(100 + n + D + block, B, H, n, D)
+    rp, col = full_csr(nb, B * H)
+    o, lse = _attn_gpu(bits, block, rp, col)
+    o_ref, lse_ref = _oracle_all(bits, block, rp, col, B, H)
+    compare_attention(o, lse, o_ref, lse_ref, f"N={n}")

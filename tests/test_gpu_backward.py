@@ -207,3 +207,16 @@ def test_full_size_sampled(name):
         keys, dk_ref, dv_ref = OB.key_block_backward(qh, kh, vh, doh, block, lrp, lcol, j_sparse[h])
         _compare([dk[0, h].float().cpu().numpy()[keys], dv[0, h].float().cpu().numpy()[keys]], [dk_ref, dv_ref],
                  f"{name} head {h} block {j_sparse[h]}", names=("dK", "dV"))
+
+
+@pytest.mark.parametrize("n", [40, 100])
+@pytest.mark.parametrize("D,block", [(128, 64), (64, 128)])
+def test_sequences_shorter_than_one_tile(n, D, block):
+    B, H = 1, 2
+    nb = -(-n // block)
+    bits = random_qkv_bf16(200 + n + D, B, H, n, D)
+    do = _dout_bits(201 + n, B, H, n, D)
+    rp, col = full_csr(nb, B * H)
+    got = _gpu(bits, do, block, rp, col)
+    ref = _oracle(bits, do, block, rp, col, B, H)
+    _compare(got, ref, f"N={n} D={D} B_s={block}")
