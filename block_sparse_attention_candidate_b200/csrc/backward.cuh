@@ -135,7 +135,8 @@ __global__ void bwd_tfill_kernel(BwdParams p) {
 //               K / V rows of the tile's kept key blocks; accumulates dQ = dS K.
 // The tile's rows are R = 128 / BS blocks; their lists (transposed CSR for
 // KV, the forward's CSR otherwise) are merged into one ascending walk, and a
-// union member's BS rows are streamed as BS / 64 steps of 64 rows.  A step's
+// union member's BS rows are streamed as BS / 64 steps of 64 rows (a 32-row
+// block as one step whose second half is masked).  A step's
 // mask bit r says whether list r holds the member: the tile rows of block r
 // get P = 0 otherwise.
 //
@@ -184,7 +185,8 @@ struct BwdTcCfg {
   static constexpr int kRows = 128;
   static constexpr int kStep = 64;
   static constexpr int kR = kRows / BS;
-  static constexpr int kSPB = BS / kStep;
+  // steps per union member; a 32-row block fills the first half of one step
+  static constexpr int kSPB = BS >= kStep ? BS / kStep : 1;
   static constexpr int kChunks = D / 64;
   static constexpr int kResBytes = kRows * D * 2;
   static constexpr int kResChunk = kRows * 128;
@@ -207,7 +209,7 @@ struct BwdTcCfg {
   __host__ __device__ static constexpr uint32_t col_x(int b) { return kXY + 128u * b; }
   __host__ __device__ static constexpr uint32_t col_y(int b) { return kXY + 128u * b + 64u; }
   static_assert(D == 64 || D == 128, "head dim");
-  static_assert(BS == 64 || BS == 128, "block size");
+  static_assert(BS == 32 || BS == 64 || BS == 128, "block size");
   static_assert(kBufs >= 2 && kXY + 128u * kBufs <= kTmemCols, "tensor memory");
   // G12(j + kBufs) waits for step j + kBufs's slot, which is freed by G34(j + kBufs - kSlots)
   static_assert(kSlots >= kBufs + 1, "slots for the MMA issue order");
@@ -472,7 +474,9 @@ __global__ void __launch_bounds__(320, 1)
       const int b = j % NB;
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (j / NB) & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
-      const bool kept = row_in && ((mt.mask >> rbit) & 1u);
+      // with 32-row blocks the step's second 32 columns belong to the next
+      // block (not this member), so that warpgroup's half is masked
+      const bool kept = row_in && ((mt.mask >> rbit) & 1u) && (BS >= 64 || g == 0);
       uint32_t xr[32], yr[32];
       tmem_ld32(taddr + lane_base + C::col_x(b) + g * 32, xr);
       tmem_ld32(taddr + lane_base + C::col_y(b) + g * 32, yr);

@@ -807,7 +807,7 @@ int dynrad_attn_backward(const void* q, const void* k, const void* v, const void
   if (B < 1 || H < 1 || N < 1 || col_cap < 0) return DYNRAD_ERR_INVALID_ARG;
   if (!(scale >= 0.0f) || !std::isfinite(scale)) return DYNRAD_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return DYNRAD_ERR_UNSUPPORTED;
-  if (block != 64 && block != 128) return DYNRAD_ERR_UNSUPPORTED;
+  if (block != 32 && block != 64 && block != 128) return DYNRAD_ERR_UNSUPPORTED;
   for (const void* ptr : {q, k, v, o, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
                           static_cast<const void*>(dv)})
     if (!aligned16(ptr)) return DYNRAD_ERR_INVALID_ARG;
@@ -872,7 +872,11 @@ int dynrad_attn_backward(const void* q, const void* k, const void* v, const void
   }
   bwd_tfill_kernel<<<wblocks, 256, 0, st>>>(bp);
   if ((rc = launch_status()) != DYNRAD_OK) return rc;
-  if (D == 128) return block == 64 ? launch_backward<128, 64>(bp, st) : launch_backward<128, 128>(bp, st);
+  if (D == 128) {
+    if (block == 32) return launch_backward<128, 32>(bp, st);
+    return block == 64 ? launch_backward<128, 64>(bp, st) : launch_backward<128, 128>(bp, st);
+  }
+  if (block == 32) return launch_backward<64, 32>(bp, st);
   return block == 64 ? launch_backward<64, 64>(bp, st) : launch_backward<64, 128>(bp, st);
 }
 

@@ -408,7 +408,8 @@ int dynrad_proxy_error(const float *lse_dense, const float *lse_kept,
  *
  *   q, k, v, o, dout  device bf16 [B, H, N, D], D = 64 or 128
  *   lse           device fp32 [B, H, N] (the forward's, natural log)
- *   block         64 or 128
+ *   block         32, 64 or 128 (at 32 each 64-row step of the tensor-core
+ *                 tiles holds one block, half the tile)
  *   row_ptr, col_idx  the forward's CSR (device int32, B*H*Nb rows, strictly
  *                 ascending block indices in [0, Nb) per row)
  *   col_cap       capacity of the transposed CSR: >= row_ptr[B*H*Nb]

@@ -273,7 +273,7 @@ def test_backward_argument_errors_before_launch():
     assert call(scale=-0.5) == abi.DYNRAD_ERR_INVALID_ARG
     assert call(scale=float("nan")) == abi.DYNRAD_ERR_INVALID_ARG
     assert call(D=96) == abi.DYNRAD_ERR_UNSUPPORTED
-    assert call(block=32) == abi.DYNRAD_ERR_UNSUPPORTED
+    assert call(block=48) == abi.DYNRAD_ERR_UNSUPPORTED
     assert call(dq=ctypes.c_void_p(0x10008)) == abi.DYNRAD_ERR_INVALID_ARG    # not 16-byte aligned
     assert call(ws=ctypes.c_void_p(0x100010)) == abi.DYNRAD_ERR_INVALID_ARG   # not 256-byte aligned
     assert call(B=300, H=300) == abi.DYNRAD_ERR_UNSUPPORTED                   # B*H > 65535

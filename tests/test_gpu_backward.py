@@ -87,7 +87,7 @@ def _random_csr(rng, BH, nb, density, empty_rows=(), dead_cols=()):
 
 
 @pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("block", [64, 128])
+@pytest.mark.parametrize("block", [32, 64, 128])
 @pytest.mark.parametrize("n", [777, 1024])
 def test_random_csr_ragged(D, block, n):
     B, H = 1, 2
@@ -143,7 +143,7 @@ def test_unsupported_block_and_capacity():
     rp = torch.tensor([0, 1], dtype=torch.int32, device="cuda")
     col = torch.zeros(1, dtype=torch.int32, device="cuda")
     with pytest.raises(abi.DynradError) as e:
-        abi.dynrad_attn_backward(q, q, q, q, lse, q, 32, rp, col)
+        abi.dynrad_attn_backward(q, q, q, q, lse, q, 48, rp, col)
     assert e.value.status == abi.DYNRAD_ERR_UNSUPPORTED
     ws = torch.empty(256, dtype=torch.uint8, device="cuda")
     with pytest.raises(abi.DynradError) as e:
@@ -210,7 +210,7 @@ def test_full_size_sampled(name):
 
 
 @pytest.mark.parametrize("n", [40, 100])
-@pytest.mark.parametrize("D,block", [(128, 64), (64, 128)])
+@pytest.mark.parametrize("D,block", [(128, 64), (64, 128), (64, 32)])
 def test_sequences_shorter_than_one_tile(n, D, block):
     B, H = 1, 2
     nb = -(-n // block)
@@ -220,3 +220,24 @@ def test_sequences_shorter_than_one_tile(n, D, block):
     got = _gpu(bits, do, block, rp, col)
     ref = _oracle(bits, do, block, rp, col, B, H)
     _compare(got, ref, f"N={n} D={D} B_s={block}")
+
+
+@pytest.mark.parametrize("mode,value", [("static", 0.25), ("dynamic", 0.8)])
+def test_tiny_workload_selected_mask(mode, value):
+    """Candidates, selection, attention and its gradient through the library on
+    the tiny workload (block 32); the oracle gets the same bf16 inputs and the
+    kept CSR."""
+    wl = WORKLOADS["tiny"]
+    g = wl.geom
+    bits = make_qkv_bf16(wl)
+    B, H, N, D = bits["q"].shape
+    do_bits = _dout_bits(301, B, H, N, D)
+    q, k, _ = gpu_inputs(bits)
+    cand = abi.dynrad_build_candidates(g)
+    rp, col, _ = abi.dynrad_select_blocks(q, k, g, cand, mode, value, scores=True)
+    torch.cuda.synchronize()
+    rp_np = rp.cpu().numpy().astype(np.int64)
+    col_np = col.cpu().numpy().astype(np.int64)[: rp_np[-1]]
+    got = _gpu(bits, do_bits, g.block, rp_np, col_np)
+    ref = _oracle(bits, do_bits, g.block, rp_np, col_np, B, H)
+    _compare(got, ref, f"tiny {mode} {value}")
