@@ -82,7 +82,7 @@ def backward_tile_fill(row_ptr: np.ndarray, col: np.ndarray, bh: int, nb: int, b
     out = {}
     for side, tile_blk, member in (("dq", qb, col), ("dkv", col, qb)):
         key = (head * nb + tile_blk // r) * nb + member
-        steps = len(np.unique(key)) * (block // 64)
+        steps = len(np.unique(key)) * max(1, block // 64)   # a 32-row block fills half a step
         out[side] = round(useful * block * block / (steps * 128.0 * 64.0), 4)
     return out
 
