@@ -192,6 +192,31 @@ def _require_cuda(*ts):
             raise ValueError("tensors must be contiguous CUDA tensors")
 
 
+_ATTN_BLOCKS = (32, 64, 128)
+
+
+def _check_attn_args(q, others, block, row_ptr, col_idx, lse=None) -> None:
+    """Host checks that keep the attention kernels inside the caller's buffers:
+    q and every tensor of `others` bf16 [B, H, N, D] of one shape, lse fp32
+    with B*H*N elements, the CSR int32 with at least B*H*Nb + 1 offsets (for
+    the block sizes the library implements; others are left to its status
+    code).  Raises ValueError."""
+    if q.dim() != 4 or q.dtype != torch.bfloat16:
+        raise ValueError("q must be a bf16 [B, H, N, D] tensor")
+    for t in others:
+        if t is not None and (t.dtype != torch.bfloat16 or t.shape != q.shape):
+            raise ValueError("q, k, v, o, dout and the gradients must be bf16 tensors of one shape")
+    B, H, N, _ = q.shape
+    if lse is not None and (lse.dtype != torch.float32 or lse.numel() != B * H * N):
+        raise ValueError("lse must be an fp32 tensor of B*H*N elements")
+    if row_ptr.dtype != torch.int32 or col_idx.dtype != torch.int32:
+        raise ValueError("row_ptr and col_idx must be int32 tensors")
+    if int(block) in _ATTN_BLOCKS:
+        need = B * H * (-(-N // int(block))) + 1
+        if row_ptr.numel() < need:
+            raise ValueError(f"row_ptr holds {row_ptr.numel()} offsets; B*H*Nb + 1 = {need} are read")
+
+
 def dynrad_num_blocks(geom) -> int:
     return int(lib().dynrad_num_blocks(ctypes.byref(make_geom(geom))))
 
@@ -277,7 +302,8 @@ def dynrad_select_blocks(q, k, geom, cand, mode, value, scores=False, buffers=No
 def dynrad_sparse_attn(q, k, v, block, row_ptr, col_idx, scale=0.0, out=None, lse=None, stream=None):
     """Stage 3.  q, k, v: bf16 [B, H, N, D] CUDA; CSR over B*H*Nb rows.
     Returns (o bf16 [B, H, N, D], lse fp32 [B, H, N])."""
-    _require_cuda(q, k, v, row_ptr, col_idx)
+    _require_cuda(q, k, v, row_ptr, col_idx, out, lse)
+    _check_attn_args(q, (k, v, out), block, row_ptr, col_idx, lse)
     B, H, N, D = q.shape
     o = torch.empty_like(q) if out is None else out
     lse_t = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
@@ -292,7 +318,8 @@ def dynrad_attn_backward(q, k, v, o, lse, dout, block, row_ptr, col_idx, scale=0
     """Gradient of stage 3 under the same CSR.  q, k, v, o, dout: bf16
     [B, H, N, D] CUDA; lse fp32 [B, H, N] from dynrad_sparse_attn.
     Returns (dq, dk, dv), bf16 [B, H, N, D]."""
-    _require_cuda(q, k, v, o, lse, dout, row_ptr, col_idx)
+    _require_cuda(q, k, v, o, lse, dout, row_ptr, col_idx, *(grads or ()))
+    _check_attn_args(q, (k, v, o, dout) + tuple(grads or ()), block, row_ptr, col_idx, lse)
     B, H, N, D = q.shape
     dq, dk, dv = grads if grads is not None else tuple(torch.empty_like(q) for _ in range(3))
     cap = col_idx.numel()

@@ -292,3 +292,38 @@ def test_backward_workspace_size_formula():
     need = B * H * (-(-N // 64) * 64) * 8 + (rows + 1) * 4 + cap * 4 + tiles * 8
     assert need <= got < need + 4 * 256
     assert L.dynrad_attn_backward_workspace_bytes(0, H, N, block, cap) == 0
+
+
+def test_attention_binding_checks_shapes_dtypes_and_csr_length():
+    import torch
+    chk = abi._check_attn_args
+    bf = torch.bfloat16
+
+    def t(*shape, dtype=bf):
+        return torch.zeros(shape, dtype=dtype)
+
+    q = t(1, 2, 1000, 64)
+    nb = -(-1000 // 64)
+    rp = t(2 * nb + 1, dtype=torch.int32)
+    col = t(5, dtype=torch.int32)
+    lse = t(1, 2, 1000, dtype=torch.float32)
+    chk(q, (q, q, None), 64, rp, col, None)                       # forward, outputs allocated
+    chk(q, (q, q, q), 64, rp, col, lse)                           # forward into caller buffers
+    chk(q, (q, q, q, q, q, q, q), 64, rp, col, lse)               # backward with caller gradients
+    chk(t(1, 1, 4096, 64), (), 32, t(129, dtype=torch.int32), col, lse.new_zeros(4096))  # one head, flat lse
+    chk(t(1, 1, 64, 64), (), 48, t(2, dtype=torch.int32), col, t(1, 1, 64, dtype=torch.float32))  # size left to the library
+    bad = [
+        lambda: chk(t(1, 2, 1000, 64, dtype=torch.float16), (), 64, rp, col),
+        lambda: chk(q, (t(1, 2, 1000, 128),), 64, rp, col),
+        lambda: chk(q, (q.float(),), 64, rp, col),
+        lambda: chk(t(2, 1000, 64), (), 64, rp, col),
+        lambda: chk(q, (), 64, rp, col, t(1, 2, 999, dtype=torch.float32)),
+        lambda: chk(q, (), 64, rp, col, t(1, 2, 1000)),
+        lambda: chk(q, (), 64, rp.long(), col),
+        lambda: chk(q, (), 64, rp, col.long()),
+        lambda: chk(q, (), 64, rp[:-1], col),                      # one offset short
+        lambda: chk(q, (), 32, rp, col),                           # block 32 reads 2 * 32 + 1 offsets
+    ]
+    for i, f in enumerate(bad):
+        with pytest.raises(ValueError):
+            f()
