@@ -83,3 +83,17 @@ def test_kept_sets_are_nested_in_tau_and_counts_match_the_z_rule():
     z = (s - mu) / (sigma + DT.EPS_Z)
     for tau in (-0.5, 0.7, 5.0):
         assert DT.kept_pairs(geom, qf, kf, 0, 3, tau, tau).sum() == max(1, int((z > tau).sum()))
+
+
+@pytest.mark.parametrize("geom", [Geometry(4, 4, 4, 8, 0.5, 2.0), Geometry(5, 3, 5, 4, 0.7, 0.3, theta_c=0.2, theta_m=0.3),
+                                  Geometry(5, 4, 4, 8, 0.5, 2.0, force_t=0)])
+@pytest.mark.parametrize("taus", [(0.5, 1.5), (2.5, 0.0), (9.0, 9.0)])
+def test_row_restricted_form_matches_the_whole_mask(geom, taus):
+    # the dense-logit per-row evaluation the full-size GPU checks use equals the
+    # rows of the pair-list construction (including the top-pair fallback)
+    qf, kf = _qk(geom, seed=4)
+    want = DT.dynamic_mask_csr(geom, qf, kf, *taus)
+    nb = geom.n_blocks
+    got = DT.dynamic_mask_rows(geom, qf, kf, taus[0], taus[1], list(range(nb)))
+    for r in range(nb):
+        np.testing.assert_array_equal(got[r], want["col"][want["row_ptr"][r]:want["row_ptr"][r + 1]])

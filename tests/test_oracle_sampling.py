@@ -148,3 +148,17 @@ def test_tiny_workload_rho_regimes_differ():
     m1 = S.sampled_mask_csr(geom, 0.9, 0.9, 1)
     m2 = S.sampled_mask_csr(geom, 0.05, 0.05, 1)
     assert m2["row_ptr"][-1] <= m1["row_ptr"][-1]
+
+
+@pytest.mark.parametrize("geom", [Geometry(4, 4, 4, 8, 0.5, 2.0), Geometry(5, 3, 5, 4, 0.7, 0.3),
+                                  Geometry(4, 4, 4, 8, 0.5, 2.0, theta_c=0.2, theta_m=0.3),
+                                  Geometry(6, 2, 5, 16, 0.4, 0.1, force_t=0)])
+@pytest.mark.parametrize("rho", [(0.3, 0.1), (0.6, 0.6)])
+def test_row_restricted_form_matches_the_whole_mask(geom, rho):
+    # the per-row evaluation the full-size GPU checks use equals the rows of the
+    # whole-matrix construction (same sample, same aggregation)
+    want = S.sampled_mask_csr(geom, rho[0], rho[1], seed=5)
+    nb = geom.n_blocks
+    got = S.sampled_mask_rows(geom, rho[0], rho[1], 5, list(range(nb)))
+    for r in range(nb):
+        np.testing.assert_array_equal(got[r], want["col"][want["row_ptr"][r]:want["row_ptr"][r + 1]])
