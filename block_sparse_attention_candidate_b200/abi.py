@@ -48,6 +48,7 @@ EXPORTED = (
     "dynrad_proxy_error",
     "dynrad_attn_backward_workspace_bytes",
     "dynrad_attn_backward",
+    "dynrad_debug_attn_stall",
 )
 
 
@@ -157,6 +158,8 @@ def lib() -> ctypes.CDLL:
         L.dynrad_attn_backward.restype = ctypes.c_int
         L.dynrad_attn_backward.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _I32, _I32, _I32, _I32, _I32, _VP, _VP,
                                            _I64, ctypes.c_float, _VP, _VP, _VP, _VP, _SZ, _VP]
+        L.dynrad_debug_attn_stall.restype = ctypes.c_int
+        L.dynrad_debug_attn_stall.argtypes = [ctypes.c_uint64, _I32]
         _lib = L
     return _lib
 
@@ -477,3 +480,10 @@ def dynrad_proxy_error(lse_dense, lse_kept, lse2_dense, lse2_kept, stream=None):
     _check(lib().dynrad_proxy_error(_ptr(lse_dense), _ptr(lse_kept), _ptr(lse2_dense), _ptr(lse2_kept),
                                     lse_dense.numel(), _ptr(out), _stream(stream)), "dynrad_proxy_error")
     return out
+
+
+def dynrad_debug_attn_stall(wait_ns: int = 0, stall_step: int = -1) -> None:
+    """Test hook of the attention forward's failure path: limit (ns) of its
+    pipeline waits and the step at which its MMA warp waits for a barrier
+    nothing completes; (0, -1) restores normal operation.  Process-wide."""
+    _check(lib().dynrad_debug_attn_stall(int(wait_ns), int(stall_step)), "dynrad_debug_attn_stall")

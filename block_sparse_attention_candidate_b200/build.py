@@ -15,7 +15,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libdynrad.so")
 SOURCES = ["dynrad.cu", "host_path.cu"]
-HEADERS = ["common.cuh", "candidates.cuh", "select.cuh", "attention.cuh", "sampling.cuh", "dyntok.cuh", "backward.cuh", "warp_mma.cuh"]
+HEADERS = ["common.cuh", "candidates.cuh", "select.cuh", "attention.cuh", "sampling.cuh", "dyntok.cuh", "backward.cuh", "warp_mma.cuh",
+           "optin.h"]
 
 
 def nvcc_path() -> str:

@@ -46,6 +46,22 @@
 
 namespace dynrad {
 
+// Developer instrumentation, compiled only with -DDYNRAD_ATTN_TRACE: lane 0 of
+// every warp of one CTA (the middle query tile of head 0) stamps clock64() at
+// fixed points of its first 64 steps into g_attn_trace[warp][step][tile][point],
+// read back with dynrad_trace_read().  Off in every normal build.
+#ifdef DYNRAD_ATTN_TRACE
+__device__ unsigned long long g_attn_trace[10][64][2][8];
+#define ATTN_TRACE(j, t, pt)                                                        \
+  do {                                                                              \
+    if (trace_cta && lane == 0 && (j) < 64) g_attn_trace[warp][(j)][(t)][(pt)] = clock64(); \
+  } while (0)
+#else
+#define ATTN_TRACE(j, t, pt) \
+  do {                       \
+  } while (0)
+#endif
+
 template <int D, int BS>
 struct AttnCfg {
   static constexpr int kTiles = 2;                   // 128-row query tiles per CTA
@@ -64,6 +80,7 @@ struct AttnCfg {
   static constexpr int kSlots = kSlotsRaw < 3 ? 3 : (kSlotsRaw > 8 ? 8 : kSlotsRaw);
   static constexpr int kSmemData = kTiles * kQTileBytes + kSlots * kTileBytes;
   static constexpr int kSmemTotal = kSmemData + kSmemCtrl + 1024;
+  static constexpr int kThreads = 320;
   static constexpr uint32_t kTmemCols = 512;
   __host__ __device__ static constexpr uint32_t col_o(int t) { return 128u * t; }
   __host__ __device__ static constexpr uint32_t col_s(int t) { return 256u + 128u * t; }
@@ -81,6 +98,9 @@ struct AttnParams {
   int N;
   int nb;
   float scale_log2;   // logit scale * log2(e)
+  uint64_t wait_ns;   // limit of the pipeline waits (kWaitLimitNs unless shortened for a test)
+  int32_t stall_step; // test hook: at this step the MMA warp waits for a barrier nothing
+                      // completes, so that wait runs out and the CTA unwinds; -1 = never
 };
 
 // One 128-key step: up to 4 kept blocks; nblk = 0 ends the walk.
@@ -98,7 +118,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 }
 
 template <int D, int BS>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(AttnCfg<D, BS>::kThreads, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -121,7 +141,8 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* s_full = meta_full + MS;       // [tile]
   uint64_t* p_full = s_full + 2;           // [tile]
   uint64_t* drain = p_full + 2;
-  StepMeta* meta = reinterpret_cast<StepMeta*>(drain + 1);
+  uint64_t* stall = drain + 1;             // never completed (failure-path tests)
+  StepMeta* meta = reinterpret_cast<StepMeta*>(stall + 1);
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(meta + MS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_s + 1);
 
@@ -130,6 +151,10 @@ __global__ void __launch_bounds__(320, 1)
   const int I0 = blockIdx.x * C::kR;
   const int q_row0 = I0 * BS;
   const int nb = p.nb;
+  const uint64_t wlim = p.wait_ns;
+#ifdef DYNRAD_ATTN_TRACE
+  const bool trace_cta = blockIdx.x == gridDim.x / 2 && blockIdx.y == 0;
+#endif
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -140,9 +165,10 @@ __global__ void __launch_bounds__(320, 1)
     for (int m = 0; m < MS; ++m) mbar_init(&meta_full[m], 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 128);
+      mbar_init(&p_full[t], 4);   // one arrival per warp of the tile's warpgroup
     }
     mbar_init(drain, 1);
+    mbar_init(stall, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -186,7 +212,7 @@ __global__ void __launch_bounds__(320, 1)
     // waits (bounded) until slot li % NS is free again
     auto slot_ready = [&](int i) -> bool {
       bool w = true;
-      if (i >= NS && lane == 0) w = mbar_wait(&slot_empty[i % NS], ((i / NS) - 1) & 1, abort_flag);
+      if (i >= NS && lane == 0) w = mbar_wait(&slot_empty[i % NS], ((i / NS) - 1) & 1, abort_flag, wlim);
       return __shfl_sync(0xffffffffu, w, 0);
     };
     for (int j = 0;; ++j) {
@@ -224,7 +250,9 @@ __global__ void __launch_bounds__(320, 1)
         st.nblk += m != INT32_MAX ? 1 : 0;
       }
       // publish the step (the walk ends with nblk = 0)
+      ATTN_TRACE(j, 0, 0);
       if (!slot_ready(li)) { ok = false; break; }
+      ATTN_TRACE(j, 0, 1);
       if (lane == 0) {
         meta[j % MS] = st;
         mbar_arrive(&meta_full[j % MS]);
@@ -269,7 +297,7 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
       const uint32_t q_base = smem_u32(q_smem);
       const uint32_t slot_base = smem_u32(slot_smem);
-      bool ok = mbar_wait(q_full, 0, abort_flag);
+      bool ok = mbar_wait(q_full, 0, abort_flag, wlim);
       bool started[2] = {false, false};   // O_t holds a P V product
       auto tile_act = [&](const StepMeta& m, int t) -> bool {
         uint32_t any = 0;
@@ -303,7 +331,7 @@ __global__ void __launch_bounds__(320, 1)
       // step 0: S_t = Q_t K(0)^T
       int j = 0;
       StepMeta cur_m;
-      if (ok && !mbar_wait(&slot_full[0], 0, abort_flag)) ok = false;
+      if (ok && !mbar_wait(&slot_full[0], 0, abort_flag, wlim)) ok = false;
       if (ok) {
         cur_m = meta[0];
         tc_fence_after();
@@ -314,19 +342,24 @@ __global__ void __launch_bounds__(320, 1)
         if (cur_m.nblk > 0) mma_commit(&slot_empty[0]);
       }
       while (ok && cur_m.nblk > 0) {
+        if (j == p.stall_step && !mbar_wait(stall, 0, abort_flag, wlim)) { ok = false; break; }
         const int iv = 2 * j + 1, ik = 2 * j + 2;   // V(j) and K(j+1) load indices
-        if (!mbar_wait(&slot_full[iv % NS], (iv / NS) & 1, abort_flag)) { ok = false; break; }
+        ATTN_TRACE(j, 0, 2);
+        if (!mbar_wait(&slot_full[iv % NS], (iv / NS) & 1, abort_flag, wlim)) { ok = false; break; }
+        ATTN_TRACE(j, 0, 3);
         StepMeta next_m;
         bool have_next = false;
         for (int t = 0; t < 2; ++t) {
           // O_t += P_t(j) V(j) once the softmax has written P_t(j)
-          if (!mbar_wait(&p_full[t], j & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&p_full[t], j & 1, abort_flag, wlim)) { ok = false; break; }
           tc_fence_after();
+          ATTN_TRACE(j, t, 0);
           if (tile_act(cur_m, t)) issue_pv(t, iv);
           if (t == 1) mma_commit(&slot_empty[iv % NS]);
           // S_t = Q_t K(j+1)^T (after the P V above in issue order)
           if (!have_next) {
-            if (!mbar_wait(&slot_full[ik % NS], (ik / NS) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&slot_full[ik % NS], (ik / NS) & 1, abort_flag, wlim)) { ok = false; break; }
+            ATTN_TRACE(j, 0, 4);
             next_m = meta[(j + 1) % MS];
             have_next = true;
             tc_fence_after();
@@ -334,6 +367,7 @@ __global__ void __launch_bounds__(320, 1)
           if (next_m.nblk > 0 && tile_act(next_m, t)) issue_qk(t, ik);
           if (t == 1 && next_m.nblk > 0) mma_commit(&slot_empty[ik % NS]);
           mma_commit(&s_full[t]);
+          ATTN_TRACE(j, t, 1);
         }
         if (!ok) break;
         cur_m = next_m;
@@ -359,11 +393,16 @@ __global__ void __launch_bounds__(320, 1)
     int j = 0;
     bool ok = true;
     for (;; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&meta_full[j % MS], (j / MS) & 1, abort_flag))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&meta_full[j % MS], (j / MS) & 1, abort_flag, wlim))) {
+        ok = false;
+        break;
+      }
       const StepMeta st = meta[j % MS];
       // S_t(j) -- or, at the end marker, completion of the last P V product
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[tile], j & 1, abort_flag))) { ok = false; break; }
+      ATTN_TRACE(j, tile, 0);
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[tile], j & 1, abort_flag, wlim))) { ok = false; break; }
       tc_fence_after();
+      ATTN_TRACE(j, tile, 1);
       if (st.nblk == 0) break;
       uint32_t tile_any = 0, row_bits = 0;
 #pragma unroll
@@ -427,6 +466,7 @@ __global__ void __launch_bounds__(320, 1)
             }
           }
         }
+        ATTN_TRACE(j, tile, 2);
         const bool active = (half_none != (1u << (C::kKeys / 64)) - 1u);
         const float m_new = active ? fmaxf(m_used, mx * c2) : m_used;
         const bool need = active && m_used != -INFINITY && m_new > m_used + 8.0f;
@@ -448,6 +488,7 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
         if (active && m_used == -INFINITY) m_used = m_new;
+        ATTN_TRACE(j, tile, 3);
         // pass 2: P over the first 64 columns of S_t; keys 64h .. 64h+63 are
         // re-read from columns 64h .. and written as bf16 pairs to columns
         // 32h .., which hold keys already consumed
@@ -499,10 +540,15 @@ __global__ void __launch_bounds__(320, 1)
         const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
         const float2 a = __fadd2_rn(a01, a23);
         l += a.x + a.y;
+        ATTN_TRACE(j, tile, 4);
         tmem_wait_st();
       }
+      // hand P_t over: every lane's stores are complete and fenced before the
+      // warp's one arrival
       tc_fence_before();
-      mbar_arrive(&p_full[tile]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[tile]);
+      ATTN_TRACE(j, tile, 5);
     }
     if (ok) {
       const bool have_o = any_pv;     // the final s_full wait covered the last P V

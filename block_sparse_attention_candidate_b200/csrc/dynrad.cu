@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -16,6 +17,7 @@
 #include "candidates.cuh"
 #include "common.cuh"
 #include "backward.cuh"
+#include "optin.h"
 #include "dyntok.cuh"
 #include "sampling.cuh"
 #include "select.cuh"
@@ -70,6 +72,23 @@ int check_geom(const dynrad_geom* g, GeomDev* out) {
 }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Grants `bytes` of dynamic shared memory to `kernel` on the current device
+// (once per device and kernel; see optin.h).
+int smem_optin(OptInTable& table, const void* kernel, int bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DYNRAD_ERR_CUDA;
+  const bool ok = table.ensure(dev, bytes, [kernel](int b) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, b) == cudaSuccess;
+  });
+  return ok ? DYNRAD_OK : DYNRAD_ERR_CUDA;
+}
+
+// Failure-path test hook of the attention kernel (dynrad_debug_attn_stall):
+// the limit of its pipeline waits (0 = the built-in limit) and the step at
+// which its MMA warp waits for a barrier nothing completes (-1 = never).
+std::atomic<uint64_t> g_attn_wait_ns{0};
+std::atomic<int32_t> g_attn_stall_step{-1};
 
 struct SelectWorkspace {
   size_t qbar, kbar, kept, partial, plan_off, plan_cnt, plan_alloc, plan_J, plan_pos, total;
@@ -152,13 +171,9 @@ int launch_attn(const void* q, const void* k, const void* v, int BH, int N, cons
   if (!encode_map(&mq, q, D, N, BH, C::kM) || !encode_map(&mk, k, D, N, BH, BS) ||
       !encode_map(&mv, v, D, N, BH, BS))
     return DYNRAD_ERR_CUDA;
-  static bool attr_set = false;  // per instantiation
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(sparse_attn_kernel<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemTotal) != cudaSuccess)
-      return DYNRAD_ERR_CUDA;
-    attr_set = true;
-  }
+  static OptInTable optin;   // per instantiation, per device
+  const int rc = smem_optin(optin, reinterpret_cast<const void*>(sparse_attn_kernel<D, BS>), C::kSmemTotal);
+  if (rc != DYNRAD_OK) return rc;
   AttnParams p;
   p.row_ptr = row_ptr;
   p.col_idx = col_idx;
@@ -167,9 +182,12 @@ int launch_attn(const void* q, const void* k, const void* v, int BH, int N, cons
   p.N = N;
   p.nb = (N + BS - 1) / BS;
   p.scale_log2 = scale * 1.4426950408889634f;
+  const uint64_t wl = g_attn_wait_ns.load(std::memory_order_relaxed);
+  p.wait_ns = wl != 0 ? wl : kWaitLimitNs;
+  p.stall_step = g_attn_stall_step.load(std::memory_order_relaxed);
   const int tiles = (p.nb + C::kR - 1) / C::kR;
   dim3 grid(tiles, BH);
-  sparse_attn_kernel<D, BS><<<grid, 320, C::kSmemTotal, st>>>(mq, mk, mv, p);
+  sparse_attn_kernel<D, BS><<<grid, C::kThreads, C::kSmemTotal, st>>>(mq, mk, mv, p);
   return launch_status();
 }
 
@@ -291,6 +309,22 @@ int dynrad_debug_exp2(const float* x, float* poly_out, float* ref_out, int64_t n
   exp2_diag_kernel<<<static_cast<unsigned>((pairs + threads - 1) / threads), threads, 0, as_stream(stream)>>>(
       x, poly_out, ref_out, n);
   return launch_status();
+}
+
+#ifdef DYNRAD_ATTN_TRACE
+// Trace builds only (see attention.cuh): copies the clock stamps to host memory.
+int dynrad_trace_read(void* host, size_t bytes) {
+  if (host == nullptr) return DYNRAD_ERR_INVALID_ARG;
+  const size_t n = bytes < sizeof(g_attn_trace) ? bytes : sizeof(g_attn_trace);
+  return cudaMemcpyFromSymbol(host, g_attn_trace, n) == cudaSuccess ? DYNRAD_OK : DYNRAD_ERR_CUDA;
+}
+#endif
+
+int dynrad_debug_attn_stall(uint64_t wait_ns, int32_t stall_step) {
+  if (stall_step < -1) return DYNRAD_ERR_INVALID_ARG;
+  g_attn_wait_ns.store(wait_ns, std::memory_order_relaxed);
+  g_attn_stall_step.store(stall_step, std::memory_order_relaxed);
+  return DYNRAD_OK;
 }
 
 int dynrad_device_status(int32_t* status_out, int32_t clear, dynrad_stream_t stream) {
@@ -759,13 +793,9 @@ template <int D, int BS, bool KV>
 int launch_bwd_tc(const BwdParams& bp, const CUtensorMap& r0, const CUtensorMap& r1, const CUtensorMap& s0,
                   const CUtensorMap& s1, const CUtensorMap& aux, cudaStream_t st) {
   using C = BwdTcCfg<D, BS, KV>;
-  static bool attr = false;   // per instantiation
-  if (!attr) {
-    if (cudaFuncSetAttribute(bwd_tc_kernel<D, BS, KV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemTotal) != cudaSuccess)
-      return DYNRAD_ERR_CUDA;
-    attr = true;
-  }
+  static OptInTable optin;   // per instantiation, per device
+  const int rc0 = smem_optin(optin, reinterpret_cast<const void*>(bwd_tc_kernel<D, BS, KV>), C::kSmemTotal);
+  if (rc0 != DYNRAD_OK) return rc0;
   const dim3 grid((bp.N + C::kRows - 1) / C::kRows, bp.BH);
   bwd_tc_kernel<D, BS, KV><<<grid, 320, C::kSmemTotal, st>>>(r0, r1, s0, s1, aux, bp);
   return launch_status();
@@ -926,10 +956,44 @@ constexpr size_t kStaticScratchBytes = static_cast<size_t>(32) << 20;  // 32 MiB
 
 static __device__ __align__(256) unsigned char g_select_scratch[kStaticScratchBytes];
 
-// Device address of g_select_scratch per device ordinal, resolved on the first
-// call on that device (the array's name in host code is only a stand-in).
+// Device address of g_select_scratch per device ordinal (the array's name in
+// host code is only a stand-in), resolved on the first call on that device and
+// again whenever the calling thread's context on it is another one than the
+// address was resolved in (a cudaDeviceReset, or a caller that made its own
+// context, loads the module anew).  Contexts are told apart by their unique
+// id, which, unlike the handle, is never reused.
+struct ScratchAddr {
+  void* addr = nullptr;
+  unsigned long long ctx_id = 0;
+};
 std::mutex g_scratch_mu;
-void* g_scratch_addr[256] = {};
+ScratchAddr g_scratch_addr[256];
+
+// Unique id of the calling thread's current context; 0 when there is none yet
+// or the driver does not provide the calls.
+unsigned long long current_context_id() {
+  using GetCurrentFn = CUresult (*)(CUcontext*);
+  using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(f);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 }  // namespace
 
@@ -948,12 +1012,16 @@ extern "C" int dynrad_select_blocks_static_scratch(
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
+    ScratchAddr& e = g_scratch_addr[dev];
+    const unsigned long long ctx = current_context_id();
+    if (e.addr == nullptr || ctx == 0 || ctx != e.ctx_id) {
+      // with this device current: the symbol lookup binds its context if needed
       void* p = nullptr;
       if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || p == nullptr) return DYNRAD_ERR_CUDA;
-      g_scratch_addr[dev] = p;
+      e.addr = p;
+      e.ctx_id = current_context_id();
     }
-    scratch = g_scratch_addr[dev];
+    scratch = e.addr;
   }
   // The scratch needs no clearing: every byte the selection reads in it is
   // written earlier in the same call.

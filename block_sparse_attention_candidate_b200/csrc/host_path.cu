@@ -104,6 +104,24 @@ struct CallObjects {
   }
 };
 
+// Joins the side streams back into the caller's stream when the call returns,
+// on every path once they exist: whatever was queued on them (copies into the
+// workspace from the caller's host buffers, copies out to them) is then ordered
+// before anything the caller queues next, even after an error return.  If an
+// event cannot be made, it falls back to waiting on the host.
+struct JoinOnReturn {
+  cudaStream_t main;
+  CallObjects* co;
+  ~JoinOnReturn() {
+    for (cudaStream_t side : {co->in, co->out}) {
+      if (side == nullptr) continue;
+      cudaEvent_t e = co->event();
+      if (e == nullptr || cudaEventRecord(e, side) != cudaSuccess || cudaStreamWaitEvent(main, e, 0) != cudaSuccess)
+        cudaStreamSynchronize(side);
+    }
+  }
+};
+
 }  // namespace
 
 extern "C" {
@@ -162,6 +180,8 @@ int dynrad_host_path(const void* q_host, const void* k_host, const void* v_host,
   const size_t row_lse = static_cast<size_t>(N) * 4;
 
   CallObjects co;
+  // declared after co: joins the side streams before co releases them
+  JoinOnReturn join{main, &co};
   if (cudaStreamCreateWithFlags(&co.in, cudaStreamNonBlocking) != cudaSuccess ||
       cudaStreamCreateWithFlags(&co.out, cudaStreamNonBlocking) != cudaSuccess)
     return DYNRAD_ERR_CUDA;
@@ -219,10 +239,7 @@ int dynrad_host_path(const void* q_host, const void* k_host, const void* v_host,
         return DYNRAD_ERR_CUDA;
     }
   }
-  // the caller's stream continues once the last copy-out is done
-  cudaEvent_t end = co.event();
-  if (end == nullptr || cudaEventRecord(end, co.out) != cudaSuccess || cudaStreamWaitEvent(main, end, 0) != cudaSuccess)
-    return DYNRAD_ERR_CUDA;
+  // the caller's stream continues once the last copy-out is done (join)
   return DYNRAD_OK;
 }
 

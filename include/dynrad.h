@@ -174,7 +174,11 @@ int dynrad_select_blocks(const void *q, const void *k, int32_t B, int32_t H,
  *   H=40 at 75,600 tokens does not); DYNRAD_ERR_INVALID_ARG for arguments the
  *   workspace size cannot be computed for; otherwise as dynrad_select_blocks.
  *   The first call on a device looks up the array's device address (with that
- *   device current); make that first call before any stream capture.
+ *   device current); make that first call before any stream capture.  The
+ *   address is looked up again when the calling thread's context on the device
+ *   is not the one it was found in (after cudaDeviceReset, or in a context the
+ *   caller created), so such a first call in the new context also belongs
+ *   before any capture.
  *   All calls on a device share the one array and it keeps the last call's
  *   contents: calls that overlap on the GPU (other streams, other host threads)
  *   race and corrupt each other's results.  Serialise them.
@@ -348,7 +352,11 @@ int dynrad_build_token_mask(const void *q, const void *k, int32_t B, int32_t H,
  * range, a geometry that does not match N, misaligned workspace),
  * DYNRAD_ERR_CAPACITY (workspace too small) -- both before any device work;
  * otherwise the errors of dynrad_select_blocks / dynrad_sparse_attn, and
- * DYNRAD_ERR_CUDA when a copy, stream or event call fails.
+ * DYNRAD_ERR_CUDA when a copy, stream or event call fails.  Such an error can
+ * come after copies of earlier chunks were queued; the call still makes
+ * `stream` wait for every copy it queued before it returns, so the rule above
+ * holds on every return: the host buffers are in use until `stream` has
+ * passed the call (their contents are then undefined for the failed run).
  * dynrad_host_path_workspace_bytes returns 0 for arguments it cannot size.
  */
 typedef struct dynrad_host_run {
@@ -447,6 +455,23 @@ int dynrad_device_status(int32_t *status_out, int32_t clear,
  */
 int dynrad_debug_exp2(const float *x, float *poly_out, float *ref_out,
                       int64_t n, dynrad_stream_t stream);
+
+/*
+ * Test hook for the attention forward's failure path (no counterpart in the
+ * paper), for launches made after the call:
+ *   wait_ns     limit, in nanoseconds of the GPU's global timer, of the
+ *               kernel's pipeline waits; 0 restores the built-in limit (2 s)
+ *   stall_step  >= 0: at that step of its walk the MMA warp of every CTA waits
+ *               for a barrier that nothing completes, so that wait runs out
+ *               after wait_ns; -1 (the default) never
+ * A wait that runs out records DYNRAD_ERR_DEVICE in the device status; every
+ * warp of the CTA unwinds, copies and tensor-core products already in flight
+ * finish (those waits always keep the full limit), tensor memory is freed and
+ * the kernel returns; the outputs of that launch are undefined.  Restore with
+ * (0, -1).  Process-wide and not synchronised with launches on other host
+ * threads: for tests only.  Errors: DYNRAD_ERR_INVALID_ARG for stall_step < -1.
+ */
+int dynrad_debug_attn_stall(uint64_t wait_ns, int32_t stall_step);
 
 /* Static string for a status code ("ok", "invalid argument", ...). */
 const char *dynrad_status_string(int32_t status);

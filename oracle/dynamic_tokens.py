@@ -24,7 +24,13 @@ Readings where the paper leaves a step open:
 * sigma is the population standard deviation over P(i, j) (divide by |P|);
   eps = 1e-6.
 * "exceeds" is strict: s~ > tau.  With sigma + eps > 0 this is
-  s > mu + tau * (sigma + eps), the form both sides evaluate.
+  s > mu + tau * (sigma + eps), the form both sides evaluate.  The pages
+  disagree here: the sentence that introduces Eq. 11 says "exceeds", while
+  Algorithm 1's dynamic-threshold step writes s~ >= tau.  The sentence beside
+  the equation is taken as the definition and the algorithm as its summary;
+  the two readings differ only on pairs whose z-score equals tau exactly,
+  which continuous scores hit with probability zero, and the GPU parity test
+  (a row between the masks at tau + 1e-3 and tau - 1e-3) accepts either.
 * The fallback pair is the one with the largest s; among equal scores the one
   with the smaller in-pair counter u * N_t + v.
 * The fallback applies per ordered frame pair (i, j), the unit the threshold

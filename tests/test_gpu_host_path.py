@@ -72,3 +72,30 @@ def test_host_path_tiny_single_chunk():
     for r, (o, lse) in zip(runs, ref):
         assert torch.equal(r["o_host"].view(torch.int16), o.view(torch.int16))
         assert torch.equal(r["lse_host"], lse)
+
+
+def test_error_after_queued_copies_leaves_the_stream_joined():
+    # the second run's rho is out of range, which dynrad_select_blocks reports at
+    # chunk 0 after the first run's copy-in and copy-out of that chunk were
+    # queued on the call's side streams; the call must still make the caller's
+    # stream wait for them, so once the stream passes the call chunk 0 of the
+    # first run is in host memory
+    wl = WORKLOADS["wan13b_480p"]
+    host = _host_inputs(wl)
+    B, H, N, D = host["q"].shape
+    runs = _runs(wl, [("static", 0.2, None), ("static", 2.0, None)], B, H, N, D)
+    ref = _device_reference(host, runs[:1])
+    chunk = 2                                     # chunk 0 = rows 0 and 1
+    ws = abi.HostPathWorkspace(B, H, N, D, runs, chunk)
+    torch.cuda.current_stream().synchronize()
+    with pytest.raises(abi.DynradError) as err:
+        abi.dynrad_host_path(host["q"], host["k"], host["v"], runs, chunk_bh=chunk, workspace=ws)
+    assert err.value.status == abi.DYNRAD_ERR_INVALID_ARG
+    passed = torch.cuda.Event()
+    passed.record()
+    passed.synchronize()
+    got_o = runs[0]["o_host"].view(B * H, N, D)[:chunk]
+    got_lse = runs[0]["lse_host"].view(B * H, N)[:chunk]
+    assert torch.equal(got_o.view(torch.int16), ref[0][0].view(B * H, N, D)[:chunk].view(torch.int16))
+    assert torch.equal(got_lse, ref[0][1].view(B * H, N)[:chunk])
+    check_device_status()

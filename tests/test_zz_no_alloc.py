@@ -35,7 +35,18 @@ def test_static_scratch_matches_workspace_entry_point(mode, value):
     check_device_status()
     n_ref = int(rp_ref[-1])
     rp_ref, col_ref, sc_ref = rp_ref.clone(), col_ref[:n_ref].clone(), sc_ref.clone()
-    for _ in range(2):                      # two calls in a row share the scratch
+    for i in range(2):                      # two checked calls share the scratch
+        if i == 1:
+            # in between, a call on other inputs (Q and K swapped, another
+            # ratio / threshold) leaves other pooled means, plan and partial
+            # sums in the scratch: a stage that read the scratch before writing
+            # it would now see stale, wrong values
+            rp2 = torch.full_like(rp_ref, -1)
+            col2 = torch.full((wl.batch * wl.heads * cand["nnz"],), -1, dtype=torch.int32, device="cuda")
+            abi.dynrad_select_blocks_static_scratch(k, q, g, cand, mode, value * 0.5, rp2, col2)
+            torch.cuda.synchronize()
+            check_device_status()
+            assert not torch.equal(rp2, rp_ref)
         rp = torch.full_like(rp_ref, -1)
         col = torch.full((wl.batch * wl.heads * cand["nnz"],), -1, dtype=torch.int32, device="cuda")
         sc = torch.full_like(sc_ref, float("nan"))
