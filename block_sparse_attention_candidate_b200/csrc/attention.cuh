@@ -305,27 +305,34 @@ __global__ void __launch_bounds__(AttnCfg<D, BS>::kThreads, 1)
         for (int b = 0; b < BPS; ++b) any |= (b < m.nblk) ? m.mask[b] : 0u;
         return ((any >> (t * C::kRT)) & kTileMask) != 0u;
       };
+      // Shared-memory descriptors: each MMA of a batch adds a constant to the
+      // batch's first descriptor (the 14-bit start-address field cannot carry:
+      // shared addresses stay below 2^18 bytes), so a batch of 8 issues costs
+      // a few integer adds beside the MMAs.
+      auto desc_add = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
+      const uint64_t qdesc0 = smem_desc_sw128(q_base, 16, 1024);
+      const uint64_t kdesc0 = smem_desc_sw128(slot_base, 16, 1024);
+      const uint64_t vdesc0 = smem_desc_sw128(slot_base, C::kKeys * 128, 1024);
       auto issue_qk = [&](int t, int i) {   // S_t = Q_t K^T, K in load slot i
-        const uint32_t qt = q_base + t * C::kQTileBytes;
-        const uint32_t kb = slot_base + (i % NS) * C::kTileBytes;
+        const uint64_t ad = desc_add(qdesc0, t * C::kQTileBytes);
+        const uint64_t bd = desc_add(kdesc0, (i % NS) * C::kTileBytes);
+        const uint32_t d = taddr + C::col_s(t);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int c = kk >> 2, off = (kk & 3) * 32;
-          const uint64_t adesc = smem_desc_sw128(qt + c * (C::kM * 128) + off, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(kb + c * (C::kKeys * 128) + off, 16, 1024);
-          mma_ss(taddr + C::col_s(t), adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+          mma_ss(d, desc_add(ad, c * (C::kM * 128) + off), desc_add(bd, c * (C::kKeys * 128) + off), idesc_qk,
+                 kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int i) {   // O_t += P_t V, V in load slot i
-        const uint32_t vb = slot_base + (i % NS) * C::kTileBytes;
+        // V tile [128 keys][D] as the MN-major B operand: 64-column chunks
+        // 128*128 bytes apart (leading offset), 8-key groups 1024 bytes apart
+        const uint64_t bd = desc_add(vdesc0, (i % NS) * C::kTileBytes);
+        const uint32_t d = taddr + C::col_o(t), a = taddr + C::col_s(t);
+        const uint32_t acc0 = started[t] ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < C::kKeys / 16; ++kk) {
-          // V tile [128 keys][D] as the MN-major B operand: 64-column chunks
-          // 128*128 bytes apart (leading offset), 8-key groups 1024 bytes apart
-          const uint64_t bdesc = smem_desc_sw128(vb + kk * 2048, C::kKeys * 128, 1024);
-          mma_ts(taddr + C::col_o(t), taddr + C::col_s(t) + kk * 8, bdesc, idesc_pv,
-                 (started[t] || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < C::kKeys / 16; ++kk)
+          mma_ts(d, a + kk * 8, desc_add(bd, kk * 2048), idesc_pv, kk > 0 ? 1u : acc0);
         started[t] = true;
       };
       // step 0: S_t = Q_t K(0)^T
@@ -344,28 +351,28 @@ __global__ void __launch_bounds__(AttnCfg<D, BS>::kThreads, 1)
       while (ok && cur_m.nblk > 0) {
         if (j == p.stall_step && !mbar_wait(stall, 0, abort_flag, wlim)) { ok = false; break; }
         const int iv = 2 * j + 1, ik = 2 * j + 2;   // V(j) and K(j+1) load indices
+        // Every wait of the step except the softmax hand-offs comes first, so
+        // that each tile's P V and Q K^T batches go out back to back: V(j),
+        // K(j+1) (or the end marker in its place; loaded steps ahead) and the
+        // next step's block list.
         ATTN_TRACE(j, 0, 2);
         if (!mbar_wait(&slot_full[iv % NS], (iv / NS) & 1, abort_flag, wlim)) { ok = false; break; }
+        if (!mbar_wait(&slot_full[ik % NS], (ik / NS) & 1, abort_flag, wlim)) { ok = false; break; }
         ATTN_TRACE(j, 0, 3);
-        StepMeta next_m;
-        bool have_next = false;
+        const StepMeta next_m = meta[(j + 1) % MS];
+        tc_fence_after();
         for (int t = 0; t < 2; ++t) {
-          // O_t += P_t(j) V(j) once the softmax has written P_t(j)
+          // O_t += P_t(j) V(j) once the softmax has written P_t(j), then
+          // S_t = Q_t K(j+1)^T (after the P V in issue order)
           if (!mbar_wait(&p_full[t], j & 1, abort_flag, wlim)) { ok = false; break; }
           tc_fence_after();
           ATTN_TRACE(j, t, 0);
           if (tile_act(cur_m, t)) issue_pv(t, iv);
-          if (t == 1) mma_commit(&slot_empty[iv % NS]);
-          // S_t = Q_t K(j+1)^T (after the P V above in issue order)
-          if (!have_next) {
-            if (!mbar_wait(&slot_full[ik % NS], (ik / NS) & 1, abort_flag, wlim)) { ok = false; break; }
-            ATTN_TRACE(j, 0, 4);
-            next_m = meta[(j + 1) % MS];
-            have_next = true;
-            tc_fence_after();
-          }
           if (next_m.nblk > 0 && tile_act(next_m, t)) issue_qk(t, ik);
-          if (t == 1 && next_m.nblk > 0) mma_commit(&slot_empty[ik % NS]);
+          if (t == 1) {
+            mma_commit(&slot_empty[iv % NS]);
+            if (next_m.nblk > 0) mma_commit(&slot_empty[ik % NS]);
+          }
           mma_commit(&s_full[t]);
           ATTN_TRACE(j, t, 1);
         }
