@@ -311,7 +311,9 @@ def workload_config(wl, args):
             "runs": [lbl for lbl, *_ in runs_of(wl)],
             "l2": "inputs larger than L2 (Q/K/V %.2f GB per step)" % (3 * wl.batch * wl.heads * g.n_tokens *
                                                                       wl.head_dim * 2 / 1e9),
-            "parallelism": ("replicas x%d (weak scaling, one layer per GPU, no collective)" % args.gpus)}
+            "parallelism": (("heads x%d (strong scaling, one layer split by heads, no collective)" % args.gpus)
+                            if getattr(args, "shard", "replicas") == "heads" and args.gpus > 1 else
+                            ("replicas x%d (weak scaling, one layer per GPU, no collective)" % args.gpus))}
 
 
 # ----------------------------------------------------------------------------
@@ -345,6 +347,9 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=3, help="query blocks per run per reference step")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling a smaller case)")
     ap.add_argument("--run", type=int, default=-1, help="time only this run of the workload")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="with several ranks: every rank runs a whole layer (replicas, weak scaling) or its "
+                         "range of the layer's heads (heads, strong scaling; no exchange is needed)")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
     if args.heads > 0:
@@ -367,10 +372,16 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", torch.cuda.current_device())
-    B, H, D, N = wl.batch, wl.heads, wl.head_dim, wl.n_tokens
+    heads_sel = None
+    if world > 1 and args.shard == "heads":
+        from block_sparse_attention_candidate_b200.sharding import head_range
+        h0, h1 = head_range(wl.heads, world, rank)
+        heads_sel = range(h0, h1)
+    B, H, D, N = wl.batch, (len(heads_sel) if heads_sel is not None else wl.heads), wl.head_dim, wl.n_tokens
 
-    # inputs: seeded synthetic layer (host, pinned) -> HBM
-    bits = make_qkv_bf16(wl)
+    # inputs: seeded synthetic layer (host, pinned) -> HBM; with head sharding
+    # only this rank's heads (each head's stream is independent of the others)
+    bits = make_qkv_bf16(wl, heads=heads_sel)
     host = {t: torch.from_numpy(bits[t].view(np.int16)).view(torch.bfloat16).pin_memory() for t in "qkv"}
     del bits
     q, k, v = (host[t].to(dev, non_blocking=False) for t in "qkv")
@@ -456,7 +467,14 @@ def main():
     attn_ms_total = float(stage_ms[:, 2].sum())
 
     peaks = load_peaks()
-    value = world * flops_step / (ms_step * 1e-3) / 1e12
+    # whole-job work: every rank's kept FLOPs (replicas: world copies of one
+    # layer; head shards: the parts of one layer)
+    flops_job = flops_step
+    if world > 1:
+        t = torch.tensor([flops_step], dtype=torch.float64, device=dev)
+        dist.all_reduce(t)
+        flops_job = float(t.item())
+    value = flops_job / (ms_step * 1e-3) / 1e12
     achieved = flops_step / (attn_ms_total * 1e-3) / 1e12
     traffic = recorded_traffic(wl.name)
 
@@ -661,7 +679,7 @@ def main():
         if st != 0:
             raise RuntimeError(f"device status after the end-to-end run: {abi.status_string(st)}")
         e2e_ms = max_over_ranks(a0.elapsed_time(a1), dev)
-        e2e = {"value": world * flops_step * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": flops_job * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms / args.steps,
                "path": f"dynrad_host_path, pinned host buffers, chunks of {args.e2e_chunk} heads"}
@@ -681,7 +699,8 @@ def main():
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "strong" if heads_sel is not None else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded correlated Fourier field + noise)",
         "config": workload_config(wl, args),
         "roofline": {"kernel": "sparse_attn_kernel", "bound": "tensor", "achieved": round(achieved, 1),

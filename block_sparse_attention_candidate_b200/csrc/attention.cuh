@@ -44,6 +44,10 @@
 
 #include "common.cuh"
 
+#ifndef DYNRAD_ATTN_POLY_PER8
+#define DYNRAD_ATTN_POLY_PER8 2
+#endif
+
 namespace dynrad {
 
 // Developer instrumentation, compiled only with -DDYNRAD_ATTN_TRACE: lane 0 of
@@ -82,6 +86,9 @@ struct AttnCfg {
   static constexpr int kSmemTotal = kSmemData + kSmemCtrl + 1024;
   static constexpr int kThreads = 320;
   static constexpr uint32_t kTmemCols = 512;
+  // pairs of exponentials (of every 8) computed on the FMA pipe
+  static constexpr int kPolyPer8 = DYNRAD_ATTN_POLY_PER8;
+  static_assert(kPolyPer8 >= 0 && kPolyPer8 <= 8, "FMA-pipe share");
   __host__ __device__ static constexpr uint32_t col_o(int t) { return 128u * t; }
   __host__ __device__ static constexpr uint32_t col_s(int t) { return 256u + 128u * t; }
   static_assert(D == 64 || D == 128, "head dim");
@@ -523,8 +530,8 @@ __global__ void __launch_bounds__(AttnCfg<D, BS>::kThreads, 1)
 #pragma unroll
               for (int q2 = 0; q2 < 32; ++q2) {
                 const float2 x = __ffma2_rn(make_float2(sv[2 * q2], sv[2 * q2 + 1]), cc, mm);
-                // one pair in four on the FMA pipe, the rest on MUFU
-                const float2 pe = (q2 & 3) == 3 ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                // kPolyPer8 pairs in eight on the FMA pipe, the rest on MUFU
+                const float2 pe = (q2 & 7) < C::kPolyPer8 ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
                 acc[q2 & 3] = __fadd2_rn(acc[q2 & 3], pe);
                 pk[q2] = pack_bf16x2(pe.x, pe.y);
               }
