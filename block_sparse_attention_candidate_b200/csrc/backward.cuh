@@ -259,8 +259,8 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int b = 0; b < NB; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 256);
-      mbar_init(&rd_done[b], 256);
+      mbar_init(&p_full[b], 8);    // one arrival per elementwise warp
+      mbar_init(&rd_done[b], 8);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -379,6 +379,7 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t idesc_g12 = idesc_bf16_f32(128, 64, false, false);
       constexpr uint32_t idesc_g34 = idesc_bf16_f32(128, D, false, true);
       const uint32_t res_base = smem_u32(res_smem);
+      auto desc_add = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
       bool ok = mbar_wait(res_full, 0, abort_flag);
       bool started = false;
       // G12 of step j into buffer j % NB; false on abort, more = false at the end marker
@@ -389,19 +390,23 @@ __global__ void __launch_bounds__(320, 1)
         if (!more) return true;
         tc_fence_after();
         const int b = j % NB;
-        const uint32_t s0 = smem_u32(slot_tile(j, 0)), s1 = smem_u32(slot_tile(j, 1));
+        // each MMA's descriptor is its batch's first one plus a constant (the
+        // 14-bit start-address field cannot carry: shared addresses < 2^18)
+        const uint64_t r0 = smem_desc_sw128(res_base, 16, 1024);
+        const uint64_t r1 = desc_add(r0, C::kResBytes);
+        const uint64_t b0 = smem_desc_sw128(smem_u32(slot_tile(j, 0)), 16, 1024);
+        const uint64_t b1 = smem_desc_sw128(smem_u32(slot_tile(j, 1)), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int c = kk >> 2, off = (kk & 3) * 32;
-          mma_ss(taddr + C::col_x(b), smem_desc_sw128(res_base + c * C::kResChunk + off, 16, 1024),
-                 smem_desc_sw128(s0 + c * C::kStepChunk + off, 16, 1024), idesc_g12, kk > 0 ? 1u : 0u);
+          mma_ss(taddr + C::col_x(b), desc_add(r0, c * C::kResChunk + off), desc_add(b0, c * C::kStepChunk + off),
+                 idesc_g12, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int c = kk >> 2, off = (kk & 3) * 32;
-          mma_ss(taddr + C::col_y(b),
-                 smem_desc_sw128(res_base + C::kResBytes + c * C::kResChunk + off, 16, 1024),
-                 smem_desc_sw128(s1 + c * C::kStepChunk + off, 16, 1024), idesc_g12, kk > 0 ? 1u : 0u);
+          mma_ss(taddr + C::col_y(b), desc_add(r1, c * C::kResChunk + off), desc_add(b1, c * C::kStepChunk + off),
+                 idesc_g12, kk > 0 ? 1u : 0u);
         }
         mma_commit(&s_full[b]);
         return true;
@@ -418,20 +423,18 @@ __global__ void __launch_bounds__(320, 1)
         const int b = j % NB;
         if (!mbar_wait(&p_full[b], (j / NB) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t s0 = smem_u32(slot_tile(j, 0)), s1 = smem_u32(slot_tile(j, 1));
+        // the step tile [64 rows][D] as the MN-major B operand: 64-column
+        // chunks kStepChunk bytes apart, 8-row groups 1024 bytes apart
+        const uint64_t t0d = smem_desc_sw128(smem_u32(slot_tile(j, 0)), C::kStepChunk, 1024);
+        const uint64_t t1d = smem_desc_sw128(smem_u32(slot_tile(j, 1)), C::kStepChunk, 1024);
 #pragma unroll
         for (int kk = 0; kk < C::kStep / 16; ++kk) {
-          // the step tile [64 rows][D] as the MN-major B operand: 64-column
-          // chunks kStepChunk bytes apart, 8-row groups 1024 bytes apart
           const uint32_t acc = (started || kk > 0) ? 1u : 0u;
           if (KV) {
-            mma_ts(taddr + C::kAcc0, taddr + C::col_x(b) + kk * 8,
-                   smem_desc_sw128(s1 + kk * 2048, C::kStepChunk, 1024), idesc_g34, acc);
-            mma_ts(taddr + C::kAcc1, taddr + C::col_y(b) + kk * 8,
-                   smem_desc_sw128(s0 + kk * 2048, C::kStepChunk, 1024), idesc_g34, acc);
+            mma_ts(taddr + C::kAcc0, taddr + C::col_x(b) + kk * 8, desc_add(t1d, kk * 2048), idesc_g34, acc);
+            mma_ts(taddr + C::kAcc1, taddr + C::col_y(b) + kk * 8, desc_add(t0d, kk * 2048), idesc_g34, acc);
           } else {
-            mma_ts(taddr + C::kAcc0, taddr + C::col_y(b) + kk * 8,
-                   smem_desc_sw128(s0 + kk * 2048, C::kStepChunk, 1024), idesc_g34, acc);
+            mma_ts(taddr + C::kAcc0, taddr + C::col_y(b) + kk * 8, desc_add(t0d, kk * 2048), idesc_g34, acc);
           }
         }
         started = true;
@@ -482,7 +485,8 @@ __global__ void __launch_bounds__(320, 1)
       tmem_ld32(taddr + lane_base + C::col_y(b) + g * 32, yr);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&rd_done[b]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rd_done[b]);
       // KV: per column pair q, q + 1 the step's {-lse2, -lse2, -D_r, -D_r};
       // padded queries carry -lse2 = -inf, so P = 0 there.  dQ side: per-row
       // constants, keys past N masked on the sequence's last step only.
@@ -525,8 +529,10 @@ __global__ void __launch_bounds__(320, 1)
       if (KV) tmem_st16(taddr + lane_base + C::col_x(b) + g * 16, pk);
       tmem_st16(taddr + lane_base + C::col_y(b) + g * 16, dk);
       tmem_wait_st();
+      // every lane's stores are complete and fenced before the warp's one arrival
       tc_fence_before();
-      mbar_arrive(&p_full[b]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[b]);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(drain, 0, abort_flag));
     if (ok) {
