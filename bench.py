@@ -42,7 +42,7 @@ from block_sparse_attention_candidate_b200.workloads import (  # noqa: E402
 METRIC = ("sparse-attn effective TFLOPS (kept blocks) at Wan-14B 720p, whole path "
           "(candidates + selection + attention) per step")
 UNIT = "TFLOP/s"
-KERNELS_PER_RUN = 9   # 3 candidate kernels, 5 selection kernels, 1 attention kernel
+KERNELS_PER_RUN = 5   # 3 candidate kernels, 1 selection kernel, 1 attention kernel
 
 
 # ----------------------------------------------------------------------------

@@ -33,6 +33,43 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// Acquire / release accesses at GPU scope, for the counters and flags that the
+// CTAs of one launch hand to each other.
+__device__ __forceinline__ int32_t ld_acquire_s32(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint64_t ld_acquire_u64(const unsigned long long* p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, uint64_t v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_release_add_s32(int32_t* p, int32_t v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Waits until *p >= target.  Bounded: when kWaitLimitNs runs out it records
+// DYNRAD_ERR_DEVICE and returns false.
+__device__ __forceinline__ bool wait_at_least(const int32_t* p, int32_t target) {
+  if (ld_acquire_s32(p) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    __nanosleep(64);
+    if (ld_acquire_s32(p) >= target) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      record_error(DYNRAD_ERR_DEVICE);
+      return false;
+    }
+  }
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

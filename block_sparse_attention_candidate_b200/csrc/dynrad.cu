@@ -28,7 +28,7 @@ namespace {
 
 constexpr int kMaxFrames = 16384;
 constexpr int kMaxBlocks = 16384;        // Nb bound of the scoring kernel's shared memory
-constexpr int kMaxRowCandidates = 1024;  // candidates per row held in a warp's registers
+constexpr int kMaxRowCandidates = 1024;  // candidates per row (a lane's kept mask covers 32 list positions)
 
 inline cudaStream_t as_stream(dynrad_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -91,26 +91,31 @@ std::atomic<uint64_t> g_attn_wait_ns{0};
 std::atomic<int32_t> g_attn_stall_step{-1};
 
 struct SelectWorkspace {
-  size_t qbar, kbar, kept, partial, plan_off, plan_cnt, plan_alloc, plan_J, plan_pos, total;
+  size_t qbar, kbar, plan_off, plan_cnt, plan_rows, plan_J, plan_pos, kept, partial, counters, zero_end, total;
 };
 
+// Counters of one stage-2 launch: ticket (8 bytes), plan_alloc, plan_done, then
+// pool_done[bh]; the range [counters, zero_end) is zeroed before each launch.
+// kept / partial serve dynamic mode's scan and compaction.
 SelectWorkspace select_layout(int64_t bh, int64_t nb, int64_t d, int64_t cand_nnz) {
   SelectWorkspace w;
   const int64_t rows = bh * nb;
+  const int64_t groups = (nb + kSelRows - 1) / kSelRows;
   const int64_t tiles = (rows + 1 + kScanTile - 1) / kScanTile;
   w.qbar = 0;
   w.kbar = align256(w.qbar + static_cast<size_t>(rows * d) * 4);
-  w.kept = align256(w.kbar + static_cast<size_t>(bh * d * padded_blocks(static_cast<int>(nb))) * 4);
-  w.partial = align256(w.kept + static_cast<size_t>(bh * cand_nnz) * 4);
   // scoring plan: per group of 8 rows, the union list and the scatter positions
   // (independent of the head; the unions' total is at most cand_nnz)
-  const int64_t groups = (nb + kSelRows - 1) / kSelRows;
-  w.plan_off = align256(w.partial + static_cast<size_t>(tiles) * 8);
+  w.plan_off = align256(w.kbar + static_cast<size_t>(rows * d) * 4);
   w.plan_cnt = align256(w.plan_off + static_cast<size_t>(groups) * 4);
-  w.plan_alloc = align256(w.plan_cnt + static_cast<size_t>(groups) * 4);
-  w.plan_J = align256(w.plan_alloc + 4);
+  w.plan_rows = align256(w.plan_cnt + static_cast<size_t>(groups) * 4);
+  w.plan_J = align256(w.plan_rows + static_cast<size_t>(groups) * 4);
   w.plan_pos = align256(w.plan_J + static_cast<size_t>(cand_nnz) * 4);
-  w.total = align256(w.plan_pos + static_cast<size_t>(cand_nnz) * kSelRows * 4);
+  w.kept = align256(w.plan_pos + static_cast<size_t>(cand_nnz) * kSelRows * 4);
+  w.partial = align256(w.kept + static_cast<size_t>(bh * cand_nnz) * 4);
+  w.counters = align256(w.partial + static_cast<size_t>(tiles) * 8);
+  w.zero_end = w.counters + 16 + static_cast<size_t>(bh) * 4;
+  w.total = align256(w.zero_end);
   return w;
 }
 
@@ -415,87 +420,80 @@ int dynrad_select_blocks(const void* q, const void* k, int32_t B, int32_t H, int
   if (workspace_bytes < w.total) return DYNRAD_ERR_CAPACITY;
   cudaStream_t st = as_stream(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* qbar = reinterpret_cast<float*>(ws + w.qbar);
-  float* kbarT = reinterpret_cast<float*>(ws + w.kbar);
-  int32_t* kept = reinterpret_cast<int32_t*>(ws + w.kept);
-  int64_t* partial = reinterpret_cast<int64_t*>(ws + w.partial);
-  const int64_t rows = bh * g.nb;
-
-  // pooling, then scoring + selection
+  const int nq = (g.nb + kSelRows - 1) / kSelRows;
+  const bool dyn = mode == DYNRAD_DYNAMIC_THRESHOLD;
+  Stage2Params sp;
+  sp.q = static_cast<const __nv_bfloat16*>(q);
+  sp.k = static_cast<const __nv_bfloat16*>(k);
+  sp.qbar = reinterpret_cast<float*>(ws + w.qbar);
+  sp.kbar = reinterpret_cast<float*>(ws + w.kbar);
+  sp.cand_row_ptr = cand_row_ptr;
+  sp.cand_col = cand_col;
+  sp.forced_lo = forced_lo;
+  sp.forced_hi = forced_hi;
+  sp.row_ptr = row_ptr;
+  sp.col_idx = col_idx;
+  sp.col_cap = col_cap;
+  sp.scores_out = scores_out;
+  sp.plan_off = reinterpret_cast<int32_t*>(ws + w.plan_off);
+  sp.plan_cnt = reinterpret_cast<int32_t*>(ws + w.plan_cnt);
+  sp.plan_J = reinterpret_cast<int32_t*>(ws + w.plan_J);
+  sp.plan_pos = reinterpret_cast<int32_t*>(ws + w.plan_pos);
+  sp.plan_rows = reinterpret_cast<int32_t*>(ws + w.plan_rows);
+  sp.ticket = reinterpret_cast<unsigned long long*>(ws + w.counters);
+  sp.plan_alloc = reinterpret_cast<int32_t*>(ws + w.counters + 8);
+  sp.plan_done = reinterpret_cast<int32_t*>(ws + w.counters + 12);
+  sp.pool_done = reinterpret_cast<int32_t*>(ws + w.counters + 16);
+  sp.kept_tmp = reinterpret_cast<int32_t*>(ws + w.kept);
+  sp.rows_bh = static_cast<int>(bh);
+  sp.cand_nnz = cand_nnz;
+  sp.N = N;
+  sp.block = g.block;
+  sp.nb = g.nb;
+  sp.nq = nq;
+  sp.max_row = (cand_max_row > 0 && cand_max_row < g.nb) ? static_cast<int>(cand_max_row) : g.nb;
+  if (sp.max_row > kMaxRowCandidates) return DYNRAD_ERR_UNSUPPORTED;
+  sp.span_cap = (kSelRows * sp.max_row + 3) & ~3;
+  sp.mode = mode;
+  sp.value = rho_or_tau;
+  sp.scale = 1.0f / std::sqrt(static_cast<float>(D));
+  const int64_t tickets = s2_tickets(nq, static_cast<int>(bh));
+  if (tickets > INT32_MAX) return DYNRAD_ERR_UNSUPPORTED;
+  size_t smem = std::max(plan_smem_bytes(g.nb), select_smem_bytes(D, sp.span_cap, dyn));
+  smem = std::max(smem, static_cast<size_t>(kSelRows) * D * 4);   // pool item's transpose tile
+  if (smem > 227 * 1024) return DYNRAD_ERR_UNSUPPORTED;
+  // list positions per lane the selection unrolls over
+  const int e = sp.max_row <= 128 ? 4 : (sp.max_row <= 256 ? 8 : (sp.max_row <= 512 ? 16 : 32));
+  const void* kern = nullptr;
+  int kid = 0;
+#define DYNRAD_S2_KERNEL(D_, DYN_, E_, ID_)                                      \
+  if (D == D_ && dyn == DYN_ && e == E_) {                                       \
+    kern = reinterpret_cast<const void*>(stage2_kernel<D_, DYN_, E_>);           \
+    kid = ID_;                                                                    \
+  }
+  DYNRAD_S2_KERNEL(64, false, 4, 0) DYNRAD_S2_KERNEL(64, false, 8, 1)
+  DYNRAD_S2_KERNEL(64, false, 16, 2) DYNRAD_S2_KERNEL(64, false, 32, 3)
+  DYNRAD_S2_KERNEL(64, true, 4, 4) DYNRAD_S2_KERNEL(64, true, 8, 5)
+  DYNRAD_S2_KERNEL(64, true, 16, 6) DYNRAD_S2_KERNEL(64, true, 32, 7)
+  DYNRAD_S2_KERNEL(128, false, 4, 8) DYNRAD_S2_KERNEL(128, false, 8, 9)
+  DYNRAD_S2_KERNEL(128, false, 16, 10) DYNRAD_S2_KERNEL(128, false, 32, 11)
+  DYNRAD_S2_KERNEL(128, true, 4, 12) DYNRAD_S2_KERNEL(128, true, 8, 13)
+  DYNRAD_S2_KERNEL(128, true, 16, 14) DYNRAD_S2_KERNEL(128, true, 32, 15)
+#undef DYNRAD_S2_KERNEL
+  if (kern == nullptr) return DYNRAD_ERR_UNSUPPORTED;
+  static OptInTable optin[16];   // per instantiation, per device
+  if ((rc = smem_optin(optin[kid], kern, static_cast<int>(smem))) != DYNRAD_OK) return rc;
+  if (cudaMemsetAsync(ws + w.counters, 0, w.zero_end - w.counters, st) != cudaSuccess) return DYNRAD_ERR_CUDA;
   {
-    Stage2Params sp;
-    sp.q = static_cast<const __nv_bfloat16*>(q);
-    sp.k = static_cast<const __nv_bfloat16*>(k);
-    sp.qbar = qbar;
-    sp.kbarT = kbarT;
-    sp.cand_row_ptr = cand_row_ptr;
-    sp.cand_col = cand_col;
-    sp.forced_lo = forced_lo;
-    sp.forced_hi = forced_hi;
-    sp.counts = row_ptr;
-    sp.kept_tmp = kept;
-    sp.scores_out = scores_out;
-    // without an export the workspace's per-candidate array holds the scores
-    // and then, row by row, the kept lists (a row's warp reads all its scores
-    // before it writes)
-    sp.scores = scores_out != nullptr ? scores_out : reinterpret_cast<float*>(kept);
-    sp.plan_off = reinterpret_cast<int32_t*>(ws + w.plan_off);
-    sp.plan_cnt = reinterpret_cast<int32_t*>(ws + w.plan_cnt);
-    sp.plan_alloc = reinterpret_cast<int32_t*>(ws + w.plan_alloc);
-    sp.plan_J = reinterpret_cast<int32_t*>(ws + w.plan_J);
-    sp.plan_pos = reinterpret_cast<int32_t*>(ws + w.plan_pos);
-    sp.rows_bh = static_cast<int>(bh);
-    sp.cand_nnz = cand_nnz;
-    sp.N = N;
-    sp.block = g.block;
-    sp.nb = g.nb;
-    sp.nbp = padded_blocks(g.nb);
-    sp.max_row = (cand_max_row > 0 && cand_max_row < g.nb) ? static_cast<int>(cand_max_row) : g.nb;
-    if (sp.max_row > kMaxRowCandidates) return DYNRAD_ERR_UNSUPPORTED;
-    sp.mode = mode;
-    sp.value = rho_or_tau;
-    sp.scale = 1.0f / std::sqrt(static_cast<float>(D));
-    const int nq = (g.nb + kSelRows - 1) / kSelRows;
-    // scoring plan (candidate CSR only, shared by all heads)
-    const size_t psmem = plan_smem_bytes(g.nb);
-    if (psmem > 227 * 1024) return DYNRAD_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(psmem)) !=
+    void* args[] = {&sp};
+    if (cudaLaunchKernel(kern, dim3(static_cast<unsigned>(tickets)), dim3(kS2Threads), args, smem, st) !=
         cudaSuccess)
       return DYNRAD_ERR_CUDA;
-    if (cudaMemsetAsync(sp.plan_alloc, 0, 4, st) != cudaSuccess) return DYNRAD_ERR_CUDA;
-    plan_kernel<<<nq, kS2Threads, psmem, st>>>(sp);
-    if ((rc = launch_status()) != DYNRAD_OK) return rc;
-    const dim3 pgrid(2 * nq, static_cast<unsigned>(bh));
-    if (D == 128)
-      pool_kernel<128><<<pgrid, kS2Threads, 0, st>>>(sp);
-    else
-      pool_kernel<64><<<pgrid, kS2Threads, 0, st>>>(sp);
-    if ((rc = launch_status()) != DYNRAD_OK) return rc;
-    // scoring: one CTA per (group of 8 rows, head), scores to their positions
-    const dim3 sgrid(nq, static_cast<unsigned>(bh));
-    if (D == 128)
-      score_kernel<128><<<sgrid, kS2Threads, 0, st>>>(sp);
-    else
-      score_kernel<64><<<sgrid, kS2Threads, 0, st>>>(sp);
-    if ((rc = launch_status()) != DYNRAD_OK) return rc;
-    // selection: one warp per row, candidates in registers
-    const unsigned rblocks = static_cast<unsigned>((rows + kSelWarps - 1) / kSelWarps);
-    const bool dyn = mode == DYNRAD_DYNAMIC_THRESHOLD;
-    const int e = sp.max_row <= 128 ? 4 : (sp.max_row <= 256 ? 8 : (sp.max_row <= 512 ? 16 : 32));
-#define DYNRAD_LAUNCH_SELECT(E_)                                               \
-  if (e == E_) {                                                               \
-    if (dyn) select_kernel<E_, true><<<rblocks, kSelWarps * 32, 0, st>>>(sp);  \
-    else select_kernel<E_, false><<<rblocks, kSelWarps * 32, 0, st>>>(sp);     \
   }
-    DYNRAD_LAUNCH_SELECT(4)
-    DYNRAD_LAUNCH_SELECT(8)
-    DYNRAD_LAUNCH_SELECT(16)
-    DYNRAD_LAUNCH_SELECT(32)
-#undef DYNRAD_LAUNCH_SELECT
+  if (dyn) {   // counts -> offsets, then the kept lists to their CSR positions
     if ((rc = launch_status()) != DYNRAD_OK) return rc;
-  }
-  // counts -> offsets, compaction
-  {
+    const int64_t rows = bh * g.nb;
+    int64_t* partial = reinterpret_cast<int64_t*>(ws + w.partial);
     const int64_t tiles = (rows + 1 + kScanTile - 1) / kScanTile;
     scan_partial_kernel<<<static_cast<unsigned>(tiles), kScanThreads, 0, st>>>(row_ptr, rows, partial);
     if ((rc = launch_status()) != DYNRAD_OK) return rc;
@@ -505,7 +503,7 @@ int dynrad_select_blocks(const void* q, const void* k, int32_t B, int32_t H, int
     cp.rows = rows;
     cp.nb = g.nb;
     cp.cand_row_ptr = cand_row_ptr;
-    cp.kept_tmp = kept;
+    cp.kept_tmp = sp.kept_tmp;
     cp.cand_nnz = cand_nnz;
     cp.col_idx = col_idx;
     cp.col_cap = col_cap;
@@ -513,8 +511,8 @@ int dynrad_select_blocks(const void* q, const void* k, int32_t B, int32_t H, int
     if ((rc = launch_status()) != DYNRAD_OK) return rc;
     const int64_t cblocks = (rows * 32 + kCompactThreads - 1) / kCompactThreads;
     compact_kernel<<<static_cast<unsigned>(cblocks), kCompactThreads, 0, st>>>(cp);
-    if ((rc = launch_status()) != DYNRAD_OK) return rc;
   }
+  if ((rc = launch_status()) != DYNRAD_OK) return rc;
   return DYNRAD_OK;
 }
 
@@ -684,6 +682,8 @@ int dynrad_build_token_mask(const void* q, const void* k, int32_t B, int32_t H, 
   if (hf > kTokMaxFusedHeads) return DYNRAD_ERR_UNSUPPORTED;
   if (g.block != 32 && g.block != 64 && g.block != 128) return DYNRAD_ERR_UNSUPPORTED;
   if (g.nt > 65535 || B > 65535) return DYNRAD_ERR_UNSUPPORTED;
+  // the aggregation keeps a frame table and one flag per candidate in default shared memory
+  if (static_cast<size_t>(g.frames) * 5 + static_cast<size_t>(g.nb) + 16 > 48 * 1024) return DYNRAD_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(B) * H * g.nb + 1 > INT32_MAX || static_cast<int64_t>(B) * cand_nnz > INT32_MAX)
     return DYNRAD_ERR_UNSUPPORTED;
   const TokWorkspace w = tok_layout(B, g.frames, g.nb, g.n, cand_nnz);
@@ -715,19 +715,43 @@ int dynrad_build_token_mask(const void* q, const void* k, int32_t B, int32_t H, 
   tp.kept_tmp = reinterpret_cast<int32_t*>(ws + w.kept);
   tp.cand_nnz = cand_nnz;
   if (cudaMemsetAsync(ws, 0, w.zero_end, st) != cudaSuccess) return DYNRAD_ERR_CUDA;
-  const size_t tsmem = static_cast<size_t>(tok_row_stride(hf * D)) * (kTokRows + kTokCols) * 2;
-  const void* tk = D == 128 ? reinterpret_cast<const void*>(dyntok_tile_kernel<128>)
-                            : reinterpret_cast<const void*>(dyntok_tile_kernel<64>);
-  if (cudaFuncSetAttribute(tk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(tsmem)) != cudaSuccess)
+  // logit tiles: tcgen05 for H_f * D <= 256, the warp-level MMA kernel above that
+  const bool use_tc = hf * D <= 256;
+  const void* tk = nullptr;
+  size_t tsmem = 0;
+  int tthreads = kTokThreads;
+  int kid = 0;
+#define DYNRAD_TOK_TC(D_, HF_, ID_)                                                     \
+  if (D == D_ && hf == HF_) {                                                           \
+    tk = reinterpret_cast<const void*>(dyntok_tc_kernel<D_, HF_>);                      \
+    tsmem = TokTcCfg<D_, HF_>::kSmemTotal;                                              \
+    tthreads = TokTcCfg<D_, HF_>::kThreads;                                             \
+    kid = ID_;                                                                          \
+  }
+#define DYNRAD_TOK_MMA(D_, HF_, ID_)                                                    \
+  if (D == D_ && hf == HF_) {                                                           \
+    tk = reinterpret_cast<const void*>(dyntok_tile_kernel<D_, HF_>);                    \
+    tsmem = tok_tile_smem(D_ * HF_);                                                    \
+    kid = ID_;                                                                          \
+  }
+  DYNRAD_TOK_TC(64, 1, 0) DYNRAD_TOK_TC(64, 2, 1) DYNRAD_TOK_TC(64, 3, 2) DYNRAD_TOK_TC(64, 4, 3)
+  DYNRAD_TOK_TC(128, 1, 4) DYNRAD_TOK_TC(128, 2, 5) DYNRAD_TOK_MMA(128, 3, 6) DYNRAD_TOK_MMA(128, 4, 7)
+#undef DYNRAD_TOK_TC
+#undef DYNRAD_TOK_MMA
+  if (tk == nullptr) return DYNRAD_ERR_UNSUPPORTED;
+  static OptInTable tok_optin[8];   // per instantiation, per device
+  if ((rc = smem_optin(tok_optin[kid], tk, static_cast<int>(tsmem))) != DYNRAD_OK) return rc;
+  CUtensorMap mq, mk;
+  if (use_tc && (!encode_map(&mq, q, D, N, B * H, 128) || !encode_map(&mk, k, D, N, B * H, 128)))
     return DYNRAD_ERR_CUDA;
   const int fp = g.frames * g.frames;
   const dim3 tgrid(fp, (g.nt + kTokRows - 1) / kTokRows, B);
   for (int pass = 0; pass < 2; ++pass) {
     tp.pass = pass;
-    if (D == 128)
-      dyntok_tile_kernel<128><<<tgrid, kTokThreads, tsmem, st>>>(tp);
-    else
-      dyntok_tile_kernel<64><<<tgrid, kTokThreads, tsmem, st>>>(tp);
+    void* args_tc[] = {&mq, &mk, &tp};
+    void* args_mma[] = {&tp};
+    if (cudaLaunchKernel(tk, tgrid, dim3(tthreads), use_tc ? args_tc : args_mma, tsmem, st) != cudaSuccess)
+      return DYNRAD_ERR_CUDA;
     if ((rc = launch_status()) != DYNRAD_OK) return rc;
     if (pass == 0) {
       const int64_t m = static_cast<int64_t>(B) * fp;
@@ -735,7 +759,7 @@ int dynrad_build_token_mask(const void* q, const void* k, int32_t B, int32_t H, 
       if ((rc = launch_status()) != DYNRAD_OK) return rc;
     }
   }
-  const size_t asmem = static_cast<size_t>(g.frames) * 5 + 16;
+  const size_t asmem = static_cast<size_t>(g.frames) * 5 + static_cast<size_t>(g.nb) + 16;
   const dim3 agrid(g.nb, B);
   if (g.block == 32) dyntok_aggregate_kernel<32><<<agrid, kTokThreads, asmem, st>>>(tp);
   else if (g.block == 64) dyntok_aggregate_kernel<64><<<agrid, kTokThreads, asmem, st>>>(tp);

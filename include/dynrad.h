@@ -110,7 +110,8 @@ int dynrad_build_candidates(const dynrad_geom *geom, int32_t *cand_row_ptr,
                             int64_t *nnz_out, int64_t *max_row_out,
                             dynrad_stream_t stream);
 
-/* Workspace bytes dynrad_select_blocks needs (pooled means + kept lists). */
+/* Workspace bytes dynrad_select_blocks needs (pooled means, scoring plan,
+ * per-call counters). */
 size_t dynrad_select_workspace_bytes(int32_t B, int32_t H, int32_t N, int32_t D,
                                      const dynrad_geom *geom, int64_t cand_nnz);
 
@@ -134,7 +135,8 @@ size_t dynrad_select_workspace_bytes(int32_t B, int32_t H, int32_t N, int32_t D,
  *   D             64 or 128
  *   cand_*, forced_*   stage-1 output for the same geometry; cand_nnz its total
  *   cand_max_row  longest candidate row (stage 1's max_row_out), or 0 for the
- *                 bound Nb; it sizes the selection's per-warp register arrays.
+ *                 bound Nb; it sizes the shared-memory score arrays of the
+ *                 selection (8 rows per CTA).
  *                 Rows of up to 1024 candidates are supported (a larger bound
  *                 returns DYNRAD_ERR_UNSUPPORTED); a row longer than the bound
  *                 is an error (device status DYNRAD_ERR_CAPACITY, row left empty)

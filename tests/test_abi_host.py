@@ -109,13 +109,14 @@ def test_workspace_size_formula():
     nnz = 331078
     ws = abi.dynrad_select_workspace_bytes(1, 40, g.n_tokens, 128, g, nnz)
     rows = 40 * g.n_blocks
-    nbp = (g.n_blocks + 31) // 32 * 32
-    # qbar [BH, Nb, D] + kbar transposed [BH, D, Nb padded to 32] (fp32) + the
-    # kept lists + scan partials + the scoring plan (per group of 8 rows: offset
-    # and size; union members and 8 scatter positions, at most cand_nnz
-    # entries), each 256-byte aligned
+    # qbar and kbar [BH, Nb, D] (fp32) + the scoring plan (per group of 8
+    # rows: offset, size and static kept count; union members and 8 scatter
+    # positions, at most cand_nnz entries) + dynamic mode's kept lists at the
+    # candidate offsets and scan partials + the launch's counters (ticket, plan
+    # counters, one per head), each region 256-byte aligned
     groups = (g.n_blocks + 7) // 8
-    need = rows * 128 * 4 + 40 * 128 * nbp * 4 + 40 * nnz * 4 + 2 * groups * 4 + 4 + nnz * 4 * 9
+    tiles = (rows + 1 + 4095) // 4096
+    need = 2 * rows * 128 * 4 + 3 * groups * 4 + nnz * 4 * 9 + 40 * nnz * 4 + tiles * 8 + 16 + 40 * 4
     assert need <= ws < need + 4096
 
 

@@ -63,7 +63,7 @@ def test_static_scratch_matches_workspace_entry_point(mode, value):
 
 
 def test_static_scratch_rejects_oversized_problems():
-    wl = WORKLOADS["wan14b_720p"]          # needs ~100 MB of scratch
+    wl = WORKLOADS["wan14b_720p"]          # needs ~60 MB of scratch
     g = wl.geom
     L = abi.lib()
     need = abi.dynrad_select_workspace_bytes(wl.batch, wl.heads, g.n_tokens, wl.head_dim, g, 331078)
