@@ -290,11 +290,12 @@ __global__ void __launch_bounds__(kTokThreads, D * HF <= 256 ? 2 : 1) dyntok_til
 // Warp roles (320 threads):
 //   warps 0-3, 4-7  epilogue: thread t of warpgroup g owns row t (TMEM lane t)
 //              and columns 64 g .. 64 g + 63 of every tile.  Pass 0 keeps, per
-//              thread, the fp64 sum and sum of squares of its row's in-band
-//              logits and the row's first maximum; pass 1 counts, per key
-//              column and query block, the logits above the threshold (a warp
-//              ballot per column, one shared-memory add per warp and query
-//              block) and adds the tile's counts to colcnt.
+//              thread, the sum and sum of squares of its row's in-band logits
+//              (fp32 over 16 columns, then fp64) and the row's first maximum;
+//              pass 1 counts, per key column and query block, the logits above
+//              the threshold (a warp ballot per column; lane l adds columns l
+//              and 32 + l to shared counters) and adds the tile's counts to
+//              colcnt.
 //   warp 8     producer: Q once, then the K tiles into a ring of two slots.
 //   warp 9     MMA issuer (one thread).
 // Every wait is bounded (common.cuh mbar_wait); a wait that runs out records
@@ -442,11 +443,13 @@ __global__ void __launch_bounds__(TokTcCfg<D, HF>::kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int u = u0 + row;
     const bool row_ok = u < nt;
-    const double thr = p.pass == 1 ? p.thr[static_cast<int64_t>(b) * F * F + pi] : 0.0;
+    // s > thr in double for a float s is s > thr rounded down to a float
+    const float thr_f = p.pass == 1 ? __double2float_rd(p.thr[static_cast<int64_t>(b) * F * F + pi]) : 0.f;
     const int I0 = (i * nt + u0) / g.block;
     const int slot = (i * nt + u) / g.block - I0;                    // this row's query block
     const int slot_first = (i * nt + u0 + (warp & 3) * 32) / g.block - I0;   // of the warp's first row
-    const bool split = __any_sync(0xffffffffu, row_ok && slot != slot_first);
+    // lanes whose row lies in the warp's first query block (the rest are in the next one)
+    const uint32_t lanes_first = __ballot_sync(0xffffffffu, !row_ok || slot == slot_first);
     // in-band columns of this row: v in [v_min, v_max]
     const int v_min = max(u - w, v_lo), v_max = min(u + w, v_hi);
     double s1 = 0.0, s2 = 0.0;
@@ -477,35 +480,45 @@ __global__ void __launch_bounds__(TokTcCfg<D, HF>::kThreads, 1)
       const int c_lo = row_ok ? v_min - vb : 1, c_hi = row_ok ? v_max - vb : 0;   // in-band columns
       uint32_t* ct = cnt + sl * (kTokSlots * C::kN);
       if (ok && p.pass == 0) {
+        // fp32 partial sums over 16 columns (two chains per sum), added to
+        // the fp64 totals once per 16 columns
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          if (c >= c_lo && c <= c_hi) {
-            const float s = sv[c] * p.inv;
-            const double sd = static_cast<double>(s);
-            s1 += sd;
-            s2 = fma(sd, sd, s2);
-            if (s > best) {   // columns ascend, so the first of equal maxima stays
-              best = s;
+        for (int c16 = 0; c16 < 64; c16 += 16) {
+          float a1[2] = {0.f, 0.f}, a2[2] = {0.f, 0.f};
+#pragma unroll
+          for (int c = c16; c < c16 + 16; ++c) {
+            const bool in = c >= c_lo && c <= c_hi;
+            const float sc = sv[c] * p.inv;
+            const float s = in ? sc : 0.f;
+            a1[c & 1] += s;
+            a2[c & 1] = fmaf(s, s, a2[c & 1]);
+            if (in && sc > best) {   // columns ascend, so the first of equal maxima stays
+              best = sc;
               best_v = vb + c;
             }
           }
+          s1 += static_cast<double>(a1[0] + a1[1]);
+          s2 += static_cast<double>(a2[0] + a2[1]);
         }
       } else if (ok) {
+        // lane l collects the counts of columns l and 32 + l from the
+        // column ballots, split between the warp's (at most two) query blocks
+        uint32_t n_lo[2] = {0u, 0u}, n_hi[2] = {0u, 0u};
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const bool kept = c >= c_lo && c <= c_hi && static_cast<double>(sv[c] * p.inv) > thr;
-          const int col = grp * 64 + c;
-          if (!split) {
-            const uint32_t bal = __ballot_sync(0xffffffffu, kept);
-            if (lane == 0 && bal != 0u) atomicAdd(&ct[slot_first * C::kN + col], static_cast<uint32_t>(__popc(bal)));
-          } else {
-            const uint32_t b0 = __ballot_sync(0xffffffffu, kept && slot == slot_first);
-            const uint32_t b1 = __ballot_sync(0xffffffffu, kept && slot != slot_first);
-            if (lane == 0) {
-              if (b0 != 0u) atomicAdd(&ct[slot_first * C::kN + col], static_cast<uint32_t>(__popc(b0)));
-              if (b1 != 0u) atomicAdd(&ct[(slot_first + 1) * C::kN + col], static_cast<uint32_t>(__popc(b1)));
-            }
+          const bool kept = c >= c_lo && c <= c_hi && sv[c] * p.inv > thr_f;
+          const uint32_t bal = __ballot_sync(0xffffffffu, kept);
+          const uint32_t lo = __popc(bal & lanes_first), hi = __popc(bal & ~lanes_first);
+          if (lane == (c & 31)) {
+            n_lo[c >> 5] = lo;
+            n_hi[c >> 5] = hi;
           }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int col = grp * 64 + h * 32 + lane;
+          if (n_lo[h] != 0u) atomicAdd(&ct[slot_first * C::kN + col], n_lo[h]);
+          if (n_hi[h] != 0u) atomicAdd(&ct[(slot_first + 1) * C::kN + col], n_hi[h]);
         }
       }
       if (p.pass == 1) {

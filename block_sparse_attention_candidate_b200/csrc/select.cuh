@@ -632,7 +632,7 @@ __device__ __forceinline__ void select_item(const Stage2Params& p, int bh, int g
     // 1 the second's.
     constexpr int kChunks = D / 4;             // float4 chunks per kbar row
     constexpr int kMine = kChunks / 2;         // chunks per thread
-    constexpr int kUnr = 4;                    // chunks per member in flight
+    constexpr int kUnr = 2;                    // chunks per member in flight
     const int U = p.plan_cnt[grp], off = p.plan_off[grp];
     const float* kb = p.kbar + static_cast<int64_t>(bh) * nb * D;
     float* exp_out = p.scores_out != nullptr ? p.scores_out + static_cast<int64_t>(bh) * p.cand_nnz : nullptr;
@@ -802,7 +802,7 @@ __device__ __forceinline__ void select_item(const Stage2Params& p, int bh, int g
 }
 
 template <int D, bool DYN, int E>
-__global__ void __launch_bounds__(kS2Threads, 3) stage2_kernel(Stage2Params p) {
+__global__ void __launch_bounds__(kS2Threads, 4) stage2_kernel(Stage2Params p) {
   extern __shared__ __align__(16) uint8_t s2_smem[];
   __shared__ long long s_ticket;
   if (threadIdx.x == 0) s_ticket = atomicAdd(p.ticket, 1ull);
