@@ -145,10 +145,11 @@ __global__ void bwd_tfill_kernel(BwdParams p) {
 //   G12  X_b = A0 B0^T, Y_b = A1 B1^T (A = resident tiles, B = the step's
 //        tiles; M = 128, N = 64, K = D).  KV: X = S^T, Y = dP^T; else X = S,
 //        Y = dP.
-//   elementwise (warps 0-7; thread = TMEM lane = tile row, warpgroup g = the
-//        32-column half g of the step): P = 2^(X c - lse2), dS = P (Y - D_r);
-//        P (KV only) and dS are written back as bf16 pairs over the first 32
-//        columns of X_b and Y_b, once both warpgroups have read their halves.
+//   elementwise (warps 0-7; thread = TMEM lane = tile row; warpgroup g takes
+//        the steps j with j mod 2 = g, so two steps' passes overlap):
+//        P = 2^(X c - lse2), dS = P (Y - D_r) over the step's 64 columns; P
+//        (KV only) and dS are written back as bf16 pairs over the first 32
+//        columns of X_b and Y_b (each warp touches only its own 32 lanes).
 //   G34  KV: dV += P^T B1, dK += dS^T B0; else dQ += dS B0 (A from tensor
 //        memory, B = the step's tile as the MN-major operand; M = 128, N = D,
 //        K = 64).
@@ -237,8 +238,7 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* s_full = slot_empty + NS;     // [NB]
   uint64_t* p_full = s_full + NB;         // [NB]
   uint64_t* drain = p_full + NB;
-  uint64_t* rd_done = drain + 1;          // [NB] both halves have read X_b, Y_b
-  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(rd_done + NB);
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_s + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -259,8 +259,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int b = 0; b < NB; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 8);    // one arrival per elementwise warp
-      mbar_init(&rd_done[b], 8);
+      mbar_init(&p_full[b], 4);    // one arrival per warp of the step's warpgroup
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -332,16 +331,22 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       if (m == INT32_MAX) {
-        // end marker: a slot with no tiles
-        if (!slot_ready(j)) { ok = false; break; }
-        if (lane == 0) {
-          BwdStepMeta* mt = reinterpret_cast<BwdStepMeta*>(slot_tail(j) + 512);
-          mt->row0 = 0;
-          mt->mask = 0u;
-          mt->end = 1;
+        // end markers: two slots with no tiles (each elementwise warpgroup
+        // meets one at the first step of its parity past the walk); row0
+        // carries the number of real steps
+        const int steps = j;
+        for (int e = 0; e < 2 && ok; ++e) {
+          if (!slot_ready(j)) { ok = false; break; }
+          if (lane == 0) {
+            BwdStepMeta* mt = reinterpret_cast<BwdStepMeta*>(slot_tail(j) + 512);
+            mt->row0 = steps;
+            mt->mask = 0u;
+            mt->end = 1;
+          }
+          __syncwarp();
+          mbar_arrive(&slot_full[j % NS]);
+          ++j;
         }
-        __syncwarp();
-        mbar_arrive(&slot_full[j % NS]);
         break;
       }
       for (int s = 0; s < C::kSPB; ++s) {
@@ -455,7 +460,7 @@ __global__ void __launch_bounds__(320, 1)
   } else {
     // ---------------------------------------------------------- elementwise
     const int t = threadIdx.x & 127;                 // tile row = TMEM lane
-    const int g = warp >> 2;                         // column half of each step
+    const int g = warp >> 2;                         // warpgroup: steps g, g + 2, ...
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int row = tile0 + t;
     const bool row_in = row < p.N;
@@ -468,66 +473,69 @@ __global__ void __launch_bounds__(320, 1)
       my_ndr = a[2];
     }
     bool ok = true;
-    int j = 0;
-    for (;; ++j) {
+    int steps = 0;   // real steps of the walk (from the end marker)
+    for (int j = g;; j += 2) {
       if (!__all_sync(0xffffffffu, mbar_wait(&slot_full[j % NS], (j / NS) & 1, abort_flag))) { ok = false; break; }
       const uint8_t* tail = slot_tail(j);
       const BwdStepMeta mt = *reinterpret_cast<const BwdStepMeta*>(tail + 512);
-      if (mt.end) break;
+      if (mt.end) {
+        steps = mt.row0;
+        break;
+      }
       const int b = j % NB;
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (j / NB) & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
-      // with 32-row blocks the step's second 32 columns belong to the next
-      // block (not this member), so that warpgroup's half is masked
-      const bool kept = row_in && ((mt.mask >> rbit) & 1u) && (BS >= 64 || g == 0);
-      uint32_t xr[32], yr[32];
-      tmem_ld32(taddr + lane_base + C::col_x(b) + g * 32, xr);
-      tmem_ld32(taddr + lane_base + C::col_y(b) + g * 32, yr);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&rd_done[b]);
       // KV: per column pair q, q + 1 the step's {-lse2, -lse2, -D_r, -D_r};
       // padded queries carry -lse2 = -inf, so P = 0 there.  dQ side: per-row
       // constants, keys past N masked on the sequence's last step only.
-      const float4* aux_s = reinterpret_cast<const float4*>(tail) + g * 16;
       const float2 cc = make_float2(c2, c2);
       const bool tail_step = !KV && mt.row0 + 64 > p.N;
-      uint32_t pk[16], dk[16];
-      if (!kept) {   // warp-uniform (the warp's 32 rows share one block) but at the sequence end
+      uint32_t pk[32], dk[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = dk[i] = 0u;
-      } else {
+      for (int h = 0; h < 2; ++h) {
+        // with 32-row blocks the step's second 32 columns belong to the next
+        // block (not this member), so that half is masked
+        const bool kept = row_in && ((mt.mask >> rbit) & 1u) && (BS >= 64 || h == 0);
+        uint32_t xr[32], yr[32];
+        tmem_ld32(taddr + lane_base + C::col_x(b) + h * 32, xr);
+        tmem_ld32(taddr + lane_base + C::col_y(b) + h * 32, yr);
+        tmem_wait_ld();
+        const float4* aux_s = reinterpret_cast<const float4*>(tail) + h * 16;
+        if (!kept) {   // warp-uniform (the warp's 32 rows share one block) but at the sequence end
 #pragma unroll
-        for (int i2 = 0; i2 < 16; ++i2) {
-          const int i = 2 * i2;   // column within the half
-          float2 l2, dd;
-          if (KV) {
-            const float4 a = aux_s[i2];
-            l2 = make_float2(a.x, a.y);
-            dd = make_float2(a.z, a.w);
-          } else {
-            l2 = make_float2(my_nl2, my_nl2);
-            dd = make_float2(my_ndr, my_ndr);
+          for (int i = 0; i < 16; ++i) pk[h * 16 + i] = dk[h * 16 + i] = 0u;
+        } else {
+#pragma unroll
+          for (int i2 = 0; i2 < 16; ++i2) {
+            const int i = 2 * i2;   // column within the half
+            float2 l2, dd;
+            if (KV) {
+              const float4 a = aux_s[i2];
+              l2 = make_float2(a.x, a.y);
+              dd = make_float2(a.z, a.w);
+            } else {
+              l2 = make_float2(my_nl2, my_nl2);
+              dd = make_float2(my_ndr, my_ndr);
+            }
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(xr[i]), __uint_as_float(xr[i + 1])), cc, l2);
+            float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            if (tail_step) {
+              const int k = mt.row0 + h * 32 + i;
+              pv.x = k < p.N ? pv.x : 0.f;
+              pv.y = k + 1 < p.N ? pv.y : 0.f;
+            }
+            const float2 y = __fadd2_rn(make_float2(__uint_as_float(yr[i]), __uint_as_float(yr[i + 1])), dd);
+            const float2 ds = __fmul2_rn(pv, y);
+            pk[h * 16 + i2] = pack_bf16x2(pv.x, pv.y);
+            dk[h * 16 + i2] = pack_bf16x2(ds.x, ds.y);
           }
-          const float2 x = __ffma2_rn(make_float2(__uint_as_float(xr[i]), __uint_as_float(xr[i + 1])), cc, l2);
-          float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          if (tail_step) {
-            const int k = mt.row0 + g * 32 + i;
-            pv.x = k < p.N ? pv.x : 0.f;
-            pv.y = k + 1 < p.N ? pv.y : 0.f;
-          }
-          const float2 y = __fadd2_rn(make_float2(__uint_as_float(yr[i]), __uint_as_float(yr[i + 1])), dd);
-          const float2 ds = __fmul2_rn(pv, y);
-          pk[i2] = pack_bf16x2(pv.x, pv.y);
-          dk[i2] = pack_bf16x2(ds.x, ds.y);
         }
       }
-      // both halves have read X_b / Y_b before either overwrites its first 32 columns
-      if (!__all_sync(0xffffffffu, mbar_wait(&rd_done[b], (j / NB) & 1, abort_flag))) { ok = false; break; }
-      tc_fence_after();
-      if (KV) tmem_st16(taddr + lane_base + C::col_x(b) + g * 16, pk);
-      tmem_st16(taddr + lane_base + C::col_y(b) + g * 16, dk);
+      // P (KV) and dS as bf16 pairs over the first 32 columns of X_b, Y_b: this
+      // warp has read all 64 columns of its own lanes, and no other warp
+      // touches them
+      if (KV) tmem_st32(taddr + lane_base + C::col_x(b), pk);
+      tmem_st32(taddr + lane_base + C::col_y(b), dk);
       tmem_wait_st();
       // every lane's stores are complete and fenced before the warp's one arrival
       tc_fence_before();
@@ -537,7 +545,7 @@ __global__ void __launch_bounds__(320, 1)
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(drain, 0, abort_flag));
     if (ok) {
       tc_fence_after();
-      const bool have = j > 0;
+      const bool have = steps > 0;
 #pragma unroll
       for (int a = 0; a < (KV ? 2 : 1); ++a) {
         // KV: a = 0 dV (scale 1), a = 1 dK (scale); else dQ (scale).  Warpgroup
