@@ -197,14 +197,19 @@ struct BwdTcCfg {
   static constexpr int kAuxBytes = KV ? 64 * 8 : 0;
   static constexpr int kSmemCtrl = 1024;
   static constexpr int kBudget = 227 * 1024 - kSmemCtrl - 1024;
-  static constexpr int kSlotsRaw = (kBudget - 2 * kResBytes) / kSlotBytes;
+  // KV: K, V resident in shared memory (the A operands of G12).  dQ side: Q,
+  // dO resident in tensor memory instead, so G12 reads only the step's tiles
+  // from shared memory and the freed space holds more slots.
+  static constexpr int kResSmem = KV ? 2 * kResBytes : 0;
+  static constexpr int kSlotsRaw = (kBudget - kResSmem) / kSlotBytes;
   static constexpr int kSlots = kSlotsRaw > 6 ? 6 : kSlotsRaw;
-  static constexpr int kSmemData = 2 * kResBytes + kSlots * kSlotBytes;
+  static constexpr int kSmemData = kResSmem + kSlots * kSlotBytes;
   static constexpr int kSmemTotal = kSmemData + kSmemCtrl + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kAcc0 = 0;
-  static constexpr uint32_t kAcc1 = D;
-  static constexpr uint32_t kXY = KV ? 2 * D : D;
+  static constexpr uint32_t kAcc1 = D;                 // KV: dK
+  static constexpr uint32_t kResA0 = D, kResA1 = D + D / 2;   // dQ side: Q, dO as bf16 pairs
+  static constexpr uint32_t kXY = 2 * D;
   // X / Y buffers: as many 128-column pairs as tensor memory holds, at most 3
   static constexpr int kBufs = (kTmemCols - kXY) / 128 > 3 ? 3 : static_cast<int>((kTmemCols - kXY) / 128);
   __host__ __device__ static constexpr uint32_t col_x(int b) { return kXY + 128u * b; }
@@ -228,8 +233,8 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ uint8_t bwd_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(bwd_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* res_smem = smem;                        // A0 at 0, A1 at kResBytes
-  uint8_t* slot_smem = smem + 2 * C::kResBytes;    // step j in slot j % NS
+  uint8_t* res_smem = smem;                        // KV: A0 at 0, A1 at kResBytes
+  uint8_t* slot_smem = smem + C::kResSmem;         // step j in slot j % NS
   uint8_t* ctrl = smem + C::kSmemData;
   uint64_t* bar = reinterpret_cast<uint64_t*>(ctrl);
   uint64_t* res_full = bar;
@@ -252,7 +257,7 @@ __global__ void __launch_bounds__(320, 1)
   auto slot_tail = [&](int j) -> uint8_t* { return slot_smem + (j % NS) * C::kSlotBytes + 2 * C::kStepBytes; };
 
   if (threadIdx.x == 0) {
-    mbar_init(res_full, 1);
+    mbar_init(res_full, KV ? 1 : 8);   // KV: the TMA transaction; dQ side: one arrival per elementwise warp
     for (int s = 0; s < NS; ++s) {
       mbar_init(&slot_full[s], 32);
       mbar_init(&slot_empty[s], 1);
@@ -298,11 +303,13 @@ __global__ void __launch_bounds__(320, 1)
       prefetch_tensormap(&tm_step0);
       prefetch_tensormap(&tm_step1);
       if (KV) prefetch_tensormap(&tm_aux);
-      mbar_arrive_expect_tx(res_full, 2 * C::kResBytes);
+      if (KV) {
+        mbar_arrive_expect_tx(res_full, 2 * C::kResBytes);
 #pragma unroll
-      for (int c = 0; c < C::kChunks; ++c) {
-        tma_load_3d(res_smem + c * C::kResChunk, &tm_res0, res_full, c * 64, tile0, bh);
-        tma_load_3d(res_smem + C::kResBytes + c * C::kResChunk, &tm_res1, res_full, c * 64, tile0, bh);
+        for (int c = 0; c < C::kChunks; ++c) {
+          tma_load_3d(res_smem + c * C::kResChunk, &tm_res0, res_full, c * 64, tile0, bh);
+          tma_load_3d(res_smem + C::kResBytes + c * C::kResChunk, &tm_res1, res_full, c * 64, tile0, bh);
+        }
       }
     }
     bool ok = true;
@@ -376,7 +383,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     if (!ok && lane == 0) {
       for (int i = (j > NS ? j - NS : 0); i < j; ++i) mbar_wait(&slot_full[i % NS], (i / NS) & 1, nullptr);
-      mbar_wait(res_full, 0, nullptr);
+      if (KV) mbar_wait(res_full, 0, nullptr);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA
@@ -404,14 +411,22 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int c = kk >> 2, off = (kk & 3) * 32;
-          mma_ss(taddr + C::col_x(b), desc_add(r0, c * C::kResChunk + off), desc_add(b0, c * C::kStepChunk + off),
-                 idesc_g12, kk > 0 ? 1u : 0u);
+          if (KV)
+            mma_ss(taddr + C::col_x(b), desc_add(r0, c * C::kResChunk + off), desc_add(b0, c * C::kStepChunk + off),
+                   idesc_g12, kk > 0 ? 1u : 0u);
+          else   // A = Q from tensor memory: 16 values of K per 8 columns
+            mma_ts(taddr + C::col_x(b), taddr + C::kResA0 + kk * 8, desc_add(b0, c * C::kStepChunk + off), idesc_g12,
+                   kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int c = kk >> 2, off = (kk & 3) * 32;
-          mma_ss(taddr + C::col_y(b), desc_add(r1, c * C::kResChunk + off), desc_add(b1, c * C::kStepChunk + off),
-                 idesc_g12, kk > 0 ? 1u : 0u);
+          if (KV)
+            mma_ss(taddr + C::col_y(b), desc_add(r1, c * C::kResChunk + off), desc_add(b1, c * C::kStepChunk + off),
+                   idesc_g12, kk > 0 ? 1u : 0u);
+          else   // A = dO from tensor memory
+            mma_ts(taddr + C::col_y(b), taddr + C::kResA1 + kk * 8, desc_add(b1, c * C::kStepChunk + off), idesc_g12,
+                   kk > 0 ? 1u : 0u);
         }
         mma_commit(&s_full[b]);
         return true;
@@ -471,6 +486,29 @@ __global__ void __launch_bounds__(320, 1)
       const float* a = p.aux + bwd_aux_index(bh, p.Np, row);
       my_nl2 = a[0];
       my_ndr = a[2];
+    }
+    if (!KV) {
+      // Q (warpgroup 0) and dO (warpgroup 1) row of this thread into tensor
+      // memory as bf16 pairs (element 2c in the low half of column c): the A
+      // operands of G12
+      const __nv_bfloat16* src = (g == 0 ? p.q : p.dout) + (static_cast<int64_t>(bh) * p.N + row) * D;
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t r[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 v4 = row_in ? reinterpret_cast<const uint4*>(src + c * 64)[i] : make_uint4(0u, 0u, 0u, 0u);
+          r[4 * i] = v4.x;
+          r[4 * i + 1] = v4.y;
+          r[4 * i + 2] = v4.z;
+          r[4 * i + 3] = v4.w;
+        }
+        tmem_st32(taddr + lane_base + (g == 0 ? C::kResA0 : C::kResA1) + c * 32, r);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(res_full);
     }
     bool ok = true;
     int steps = 0;   // real steps of the walk (from the end marker)
