@@ -160,9 +160,10 @@ __global__ void bwd_tfill_kernel(BwdParams p) {
 // Warp roles (320 threads): warps 0-7 elementwise and epilogue, warp 8
 // producer (list walk, TMA loads into a ring of slots, per-query lse2 / D_r of
 // the step for KV), warp 9 MMA issuer.  Tensor memory (512 columns): acc0 at 0
-// (dV or dQ), acc1 at D (dK, KV only), then X_b at base + 128 b and Y_b at
-// base + 128 b + 64 (base = 2D for KV, D otherwise).  Every wait is bounded
-// (common.cuh).
+// (dV or dQ); KV: acc1 (dK) at D; dQ side: Q at D and dO at 3D / 2 as bf16
+// pairs (G12's A operands, written by the elementwise warps); then X_b at
+// 2D + 128 b and Y_b at 2D + 128 b + 64.  KV keeps K, V in shared memory (G12
+// reads them from there).  Every wait is bounded (common.cuh).
 // ----------------------------------------------------------------------------
 // 2-D tiled TMA load (non-multicast) of the per-row (-lse2, -D_r) pairs.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
