@@ -273,8 +273,10 @@ int dynrad_build_sampled_mask(const dynrad_geom *geom, double rho1, double rho2,
  *
  * For every candidate token pair (u, v) of an ordered frame pair (i, j) at
  * t >= 2 kept by the split rule: s = (1/hf) sum_{h < hf} q_u^h . k_v^h /
- * sqrt(D) over the FIRST hf heads (fp32 FMAs, fixed order); per frame pair,
- * mu and the population sigma of s over P(i, j) (fp64 sums); the pair is kept
+ * sqrt(D) over the FIRST hf heads (bf16 tensor-core products, fp32
+ * accumulation in a fixed order); per frame pair, mu and the population sigma
+ * of s over P(i, j) (fp32 partial sums of at most 16 logits, added in fp64);
+ * the pair is kept
  * when (s - mu) / (sigma + 1e-6) > tau, tau = tau1 when L(t) >= block, tau2
  * otherwise; if none passes, the pair with the largest s (smallest u*N_t + v
  * among equals) is kept.  Pairs at t <= 1 are all kept.  Kept links are
@@ -294,7 +296,8 @@ int dynrad_build_sampled_mask(const dynrad_geom *geom, double rho1, double rho2,
  *                 (B, N, geom, cand_nnz) bytes (holds a B x Nb x N counter
  *                 array: ~360 MB per batch element at 75,600 tokens, block 64)
  * Errors: DYNRAD_ERR_INVALID_ARG / UNSUPPORTED / CAPACITY before any launch
- * (null pointer, hf out of range, non-finite tau, D, block, N_t > 65535);
+ * (null pointer, hf out of range, non-finite tau, D, block, N_t > 65535,
+ * 5 * frames + Nb > 49,136);
  * a col_idx capacity exceeded on the device is recorded in the device status.
  */
 size_t dynrad_token_mask_workspace_bytes(int32_t B, int32_t N,
