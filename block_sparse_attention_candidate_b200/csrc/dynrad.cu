@@ -745,7 +745,16 @@ int dynrad_build_token_mask(const void* q, const void* k, int32_t B, int32_t H, 
   if (use_tc && (!encode_map(&mq, q, D, N, B * H, 128) || !encode_map(&mk, k, D, N, B * H, 128)))
     return DYNRAD_ERR_CUDA;
   const int fp = g.frames * g.frames;
-  const dim3 tgrid(fp, (g.nt + kTokRows - 1) / kTokRows, B);
+  dim3 tgrid(fp, (g.nt + kTokRows - 1) / kTokRows, B);
+  if (use_tc) {   // persistent: one CTA per SM over the (frame pair, 128 rows, batch) units
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+      return DYNRAD_ERR_CUDA;
+    const int64_t units = static_cast<int64_t>(B) * fp * ((g.nt + 127) / 128);
+    if (units > INT32_MAX) return DYNRAD_ERR_UNSUPPORTED;
+    tgrid = dim3(static_cast<unsigned>(std::min<int64_t>(units, sms)), 1, 1);
+  }
   for (int pass = 0; pass < 2; ++pass) {
     tp.pass = pass;
     void* args_tc[] = {&mq, &mk, &tp};

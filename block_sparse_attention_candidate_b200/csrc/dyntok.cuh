@@ -280,8 +280,8 @@ __global__ void __launch_bounds__(kTokThreads, D * HF <= 256 ? 2 : 1) dyntok_til
 // The same logit tiles on the 5th-generation tensor cores, for dot-product
 // lengths H_f * D <= 256 (the usual two fused heads of 128 dimensions).
 //
-// One CTA per (frame pair, 128 rows u, batch) walks its band in 128-column
-// tiles: S = Q_u K_v^T, 128 x 128 x (H_f * D), bf16 operands staged by TMA
+// Persistent CTAs walk work units (frame pair, 128 rows u, batch); a unit is
+// its band in 128-column tiles: S = Q_u K_v^T, 128 x 128 x (H_f * D), bf16 operands staged by TMA
 // (128-byte swizzle, one 64-column chunk per head half), fp32 accumulation in
 // tensor memory, double-buffered so the product of tile j + 1 runs while tile
 // j is read out.  The k order of the accumulation is fixed, so both passes see
@@ -312,7 +312,7 @@ struct TokTcCfg {
   static constexpr int kSlots = 2;
   static constexpr int kSmemData = kQBytes + kSlots * kKBytes;
   static constexpr int kCntWords = 2 * kTokSlots * kN;   // [tile parity][query block][column]
-  static constexpr int kSmemCtrl = 320 + kCntWords * 4;   // barriers, reductions, counters
+  static constexpr int kSmemCtrl = 512 + kCntWords * 4;   // barriers, reductions, counters
   static constexpr int kSmemTotal = kSmemData + kSmemCtrl + 1024;   // 1024: manual alignment
   static constexpr int kThreads = 320;
   static constexpr uint32_t kTmemCols = 256;         // two 128-column S buffers
@@ -320,6 +320,39 @@ struct TokTcCfg {
   static_assert(kSmemTotal <= 227 * 1024, "shared memory");
 };
 
+// One work unit of the tensor-core tile kernel: (frame pair, 128 query rows,
+// batch element).  Units where the pair is not scored (t < 2, or dropped by
+// the split rule) have no tiles; every role skips them alike.
+struct TokUnit {
+  int pi, i, j, u0, b, w, v_lo, v_hi, ntile;
+};
+
+__device__ __forceinline__ TokUnit tok_unit(const GeomDev& g, int u, int nchunks, int rows, int cols) {
+  TokUnit x;
+  const int F = g.frames, nt = g.nt;
+  const int per_b = F * F * nchunks;
+  x.b = u / per_b;
+  const int r = u - x.b * per_b;
+  x.pi = r / nchunks;
+  x.u0 = (r - x.pi * nchunks) * rows;
+  x.i = x.pi / F;
+  x.j = x.pi - x.i * F;
+  const int t = x.i > x.j ? x.i - x.j : x.j - x.i;
+  x.ntile = 0;
+  x.w = 0;
+  x.v_lo = x.v_hi = 0;
+  if (t >= 2 && x.u0 < nt && pair_retained(g, t)) {
+    x.w = window_width(g, t);
+    x.v_lo = max(x.u0 - x.w, 0);
+    x.v_hi = min(x.u0 + rows - 1 + x.w, nt - 1);
+    x.ntile = (x.v_hi - x.v_lo + cols) / cols;
+  }
+  return x;
+}
+
+// Persistent: CTA c takes units c, c + gridDim.x, ...; tensor memory, the
+// barriers and the K ring live across units, so the next unit's Q and K loads
+// run while the current unit's last tiles are read out.
 template <int D, int HF>
 __global__ void __launch_bounds__(TokTcCfg<D, HF>::kThreads, 1)
     dyntok_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -328,15 +361,8 @@ __global__ void __launch_bounds__(TokTcCfg<D, HF>::kThreads, 1)
   extern __shared__ uint8_t tok_tc_raw[];
   const GeomDev& g = p.g;
   const int F = g.frames, nt = g.nt;
-  const int pi = blockIdx.x, b = blockIdx.z;
-  const int i = pi / F, j = pi % F;
-  const int t = i > j ? i - j : j - i;
-  if (t < 2 || !pair_retained(g, t)) return;
-  const int w = window_width(g, t);
-  const int u0 = blockIdx.y * C::kM;
-  if (u0 >= nt) return;
-  const int v_lo = max(u0 - w, 0), v_hi = min(u0 + C::kM - 1 + w, nt - 1);
-  const int ntile = (v_hi - v_lo + C::kN) / C::kN;
+  const int nchunks = (nt + C::kM - 1) / C::kM;
+  const int nunits = p.B * F * F * nchunks;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(tok_tc_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* q_smem = smem;
@@ -344,20 +370,22 @@ __global__ void __launch_bounds__(TokTcCfg<D, HF>::kThreads, 1)
   uint8_t* ctrl = smem + C::kSmemData;
   uint64_t* bar = reinterpret_cast<uint64_t*>(ctrl);
   uint64_t* q_full = bar;
-  uint64_t* k_full = bar + 1;      // [2]
-  uint64_t* k_empty = bar + 3;     // [2]
-  uint64_t* s_full = bar + 5;      // [2]
-  uint64_t* s_empty = bar + 7;     // [2]
-  uint64_t* drain = bar + 9;
-  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(bar + 10);
+  uint64_t* q_empty = bar + 1;     // a unit's products are done with Q
+  uint64_t* k_full = bar + 2;      // [2]
+  uint64_t* k_empty = bar + 4;     // [2]
+  uint64_t* s_full = bar + 6;      // [2]
+  uint64_t* s_empty = bar + 8;     // [2]
+  uint64_t* drain = bar + 10;
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(bar + 11);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_s + 1);
-  double* red_d = reinterpret_cast<double*>(ctrl + 128);                  // [2][8]
-  unsigned long long* red_b = reinterpret_cast<unsigned long long*>(ctrl + 256);   // [8]
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(ctrl + 320);               // [2][kTokSlots][kN]
+  double* red_d = reinterpret_cast<double*>(ctrl + 128);                   // [2 parities][2][8]
+  unsigned long long* red_b = reinterpret_cast<unsigned long long*>(ctrl + 384);   // [2 parities][8]
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(ctrl + 512);                // [2][kTokSlots][kN]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
@@ -383,28 +411,35 @@ __global__ void __launch_bounds__(TokTcCfg<D, HF>::kThreads, 1)
     if (lane == 0) {
       prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_k);
-      mbar_arrive_expect_tx(q_full, C::kQBytes);
-#pragma unroll
-      for (int c = 0; c < C::kChunks; ++c)
-        tma_load_3d(q_smem + c * (C::kM * 128), &tm_q, q_full, (c % C::kChunksPerHead) * 64, i * nt + u0,
-                    b * p.H + c / C::kChunksPerHead);
-      int issued = 0;
-      for (int jt = 0; jt < ntile; ++jt) {
-        const int sl = jt & 1;
-        if (jt >= 2 && !mbar_wait(&k_empty[sl], ((jt >> 1) - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&k_full[sl], C::kKBytes);
-        const int v0 = v_lo + jt * C::kN;
+      int gt = 0, ul = 0;   // K tiles and units issued
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+        const TokUnit x = tok_unit(g, u, nchunks, C::kM, C::kN);
+        if (x.ntile == 0) continue;
+        if (ul > 0 && !mbar_wait(q_empty, (ul - 1) & 1, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(q_full, C::kQBytes);
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(k_smem + sl * C::kKBytes + c * (C::kN * 128), &tm_k, &k_full[sl],
-                      (c % C::kChunksPerHead) * 64, j * nt + v0, b * p.H + c / C::kChunksPerHead);
-        issued = jt + 1;
+          tma_load_3d(q_smem + c * (C::kM * 128), &tm_q, q_full, (c % C::kChunksPerHead) * 64, x.i * nt + x.u0,
+                      x.b * p.H + c / C::kChunksPerHead);
+        ++ul;
+        for (int jt = 0; jt < x.ntile; ++jt) {
+          const int sl = gt & 1;
+          if (gt >= 2 && !mbar_wait(&k_empty[sl], ((gt >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&k_full[sl], C::kKBytes);
+          const int v0 = x.v_lo + jt * C::kN;
+#pragma unroll
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(k_smem + sl * C::kKBytes + c * (C::kN * 128), &tm_k, &k_full[sl],
+                        (c % C::kChunksPerHead) * 64, x.j * nt + v0, x.b * p.H + c / C::kChunksPerHead);
+          ++gt;
+        }
       }
-      if (issued < ntile) {
+      if (!ok) {
         // unwinding: the copies already issued land before shared memory is
         // given back (bounded; ignores the abort flag)
-        mbar_wait(q_full, 0, nullptr);
-        for (int jt = issued > 2 ? issued - 2 : 0; jt < issued; ++jt) mbar_wait(&k_full[jt & 1], (jt >> 1) & 1, nullptr);
+        if (ul > 0) mbar_wait(q_full, (ul - 1) & 1, nullptr);
+        for (int k = gt > 2 ? gt - 2 : 0; k < gt; ++k) mbar_wait(&k_full[k & 1], (k >> 1) & 1, nullptr);
       }
     }
     __syncwarp();
@@ -415,21 +450,31 @@ __global__ void __launch_bounds__(TokTcCfg<D, HF>::kThreads, 1)
       auto desc_add = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (bytes >> 4); };
       const uint64_t qdesc0 = smem_desc_sw128(smem_u32(q_smem), 16, 1024);
       const uint64_t kdesc0 = smem_desc_sw128(smem_u32(k_smem), 16, 1024);
-      bool ok = mbar_wait(q_full, 0, abort_flag);
-      for (int jt = 0; ok && jt < ntile; ++jt) {
-        const int sl = jt & 1;
-        if (!mbar_wait(&k_full[sl], (jt >> 1) & 1, abort_flag)) { ok = false; break; }
-        if (jt >= 2 && !mbar_wait(&s_empty[sl], ((jt >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint64_t bd = desc_add(kdesc0, sl * C::kKBytes);
+      int gt = 0, ul = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < nunits; u += gridDim.x) {
+        const TokUnit x = tok_unit(g, u, nchunks, C::kM, C::kN);
+        if (x.ntile == 0) continue;
+        if (!mbar_wait(q_full, ul & 1, abort_flag)) { ok = false; break; }
+        for (int jt = 0; jt < x.ntile; ++jt) {
+          const int sl = gt & 1;
+          if (!mbar_wait(&k_full[sl], (gt >> 1) & 1, abort_flag)) { ok = false; break; }
+          if (gt >= 2 && !mbar_wait(&s_empty[sl], ((gt >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t bd = desc_add(kdesc0, sl * C::kKBytes);
 #pragma unroll
-        for (int kk = 0; kk < C::kX / 16; ++kk) {
-          const int c = kk >> 2, off = (kk & 3) * 32;
-          mma_ss(taddr + sl * C::kN, desc_add(qdesc0, c * (C::kM * 128) + off), desc_add(bd, c * (C::kN * 128) + off),
-                 idesc, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < C::kX / 16; ++kk) {
+            const int c = kk >> 2, off = (kk & 3) * 32;
+            mma_ss(taddr + sl * C::kN, desc_add(qdesc0, c * (C::kM * 128) + off),
+                   desc_add(bd, c * (C::kN * 128) + off), idesc, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&k_empty[sl]);
+          mma_commit(&s_full[sl]);
+          ++gt;
         }
-        mma_commit(&k_empty[sl]);
-        mma_commit(&s_full[sl]);
+        if (!ok) break;
+        mma_commit(q_empty);   // the unit's products are done with Q
+        ++ul;
       }
       // all issued tensor-core work finished before tensor memory is released
       mma_commit(drain);
@@ -441,138 +486,149 @@ __global__ void __launch_bounds__(TokTcCfg<D, HF>::kThreads, 1)
     const int grp = warp >> 2;                     // column half
     const int row = (warp & 3) * 32 + lane;        // TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int u = u0 + row;
-    const bool row_ok = u < nt;
-    // s > thr in double for a float s is s > thr rounded down to a float
-    const float thr_f = p.pass == 1 ? __double2float_rd(p.thr[static_cast<int64_t>(b) * F * F + pi]) : 0.f;
-    const int I0 = (i * nt + u0) / g.block;
-    const int slot = (i * nt + u) / g.block - I0;                    // this row's query block
-    const int slot_first = (i * nt + u0 + (warp & 3) * 32) / g.block - I0;   // of the warp's first row
-    // lanes whose row lies in the warp's first query block (the rest are in the next one)
-    const uint32_t lanes_first = __ballot_sync(0xffffffffu, !row_ok || slot == slot_first);
-    // in-band columns of this row: v in [v_min, v_max]
-    const int v_min = max(u - w, v_lo), v_max = min(u + w, v_hi);
-    double s1 = 0.0, s2 = 0.0;
-    float best = -INFINITY;
-    int best_v = -1;
-    // After a failed wait the warp keeps stepping through the tiles without
-    // work, so every warp of the warpgroup reaches the same named barriers.
+    // After a failed wait the warps keep stepping through the units and tiles
+    // without work, so every warp reaches the same named barriers.
     bool ok = true;
-    for (int jt = 0; jt < ntile; ++jt) {
-      const int sl = jt & 1;
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sl], (jt >> 1) & 1, abort_flag));
-      float sv[64];
-      if (ok) {
-        tc_fence_after();
+    int gt = 0, ul = 0;
+    for (int uu = blockIdx.x; uu < nunits; uu += gridDim.x) {
+      const TokUnit x = tok_unit(g, uu, nchunks, C::kM, C::kN);
+      if (x.ntile == 0) continue;
+      const int u = x.u0 + row;
+      const bool row_ok = u < nt;
+      // s > thr in double for a float s is s > thr rounded down to a float
+      const float thr_f =
+          p.pass == 1 ? __double2float_rd(p.thr[static_cast<int64_t>(x.b) * F * F + x.pi]) : 0.f;
+      const int I0 = (x.i * nt + x.u0) / g.block;
+      const int slot = (x.i * nt + u) / g.block - I0;                      // this row's query block
+      const int slot_first = (x.i * nt + x.u0 + (warp & 3) * 32) / g.block - I0;   // of the warp's first row
+      // lanes whose row lies in the warp's first query block (the rest are in the next one)
+      const uint32_t lanes_first = __ballot_sync(0xffffffffu, !row_ok || slot == slot_first);
+      // in-band columns of this row: v in [v_min, v_max]
+      const int v_min = max(u - x.w, x.v_lo), v_max = min(u + x.w, x.v_hi);
+      double s1 = 0.0, s2 = 0.0;
+      float best = -INFINITY;
+      int best_v = -1;
+      for (int jt = 0; jt < x.ntile; ++jt, ++gt) {
+        const int sl = gt & 1;
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sl], (gt >> 1) & 1, abort_flag));
+        const int vb = x.v_lo + jt * C::kN + grp * 64;   // column 0 of this thread's half
+        const int c_lo = row_ok ? v_min - vb : 1, c_hi = row_ok ? v_max - vb : 0;   // in-band columns
+        float sv[64];
+        if (ok) {
+          tc_fence_after();
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t r[32];
-          tmem_ld32(taddr + lane_base + sl * C::kN + grp * 64 + h * 32, r);
+          for (int h = 0; h < 2; ++h) {
+            uint32_t r[32];
+            tmem_ld32(taddr + lane_base + sl * C::kN + grp * 64 + h * 32, r);
 #pragma unroll
-          for (int x = 0; x < 32; ++x) sv[h * 32 + x] = __uint_as_float(r[x]);
+            for (int q = 0; q < 32; ++q) sv[h * 32 + q] = __uint_as_float(r[q]);
+          }
+          tmem_wait_ld();
         }
-        tmem_wait_ld();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[sl]);
-      const int vb = v_lo + jt * C::kN + grp * 64;   // column 0 of this thread's half
-      const int c_lo = row_ok ? v_min - vb : 1, c_hi = row_ok ? v_max - vb : 0;   // in-band columns
-      uint32_t* ct = cnt + sl * (kTokSlots * C::kN);
-      if (ok && p.pass == 0) {
-        // fp32 partial sums over 16 columns (two chains per sum), added to
-        // the fp64 totals once per 16 columns
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[sl]);
+        uint32_t* ct = cnt + sl * (kTokSlots * C::kN);
+        if (ok && p.pass == 0) {
+          // fp32 partial sums over 16 columns (two chains per sum), added to
+          // the fp64 totals once per 16 columns
 #pragma unroll
-        for (int c16 = 0; c16 < 64; c16 += 16) {
-          float a1[2] = {0.f, 0.f}, a2[2] = {0.f, 0.f};
+          for (int c16 = 0; c16 < 64; c16 += 16) {
+            float a1[2] = {0.f, 0.f}, a2[2] = {0.f, 0.f};
 #pragma unroll
-          for (int c = c16; c < c16 + 16; ++c) {
-            const bool in = c >= c_lo && c <= c_hi;
-            const float sc = sv[c] * p.inv;
-            const float s = in ? sc : 0.f;
-            a1[c & 1] += s;
-            a2[c & 1] = fmaf(s, s, a2[c & 1]);
-            if (in && sc > best) {   // columns ascend, so the first of equal maxima stays
-              best = sc;
-              best_v = vb + c;
+            for (int c = c16; c < c16 + 16; ++c) {
+              const bool in = c >= c_lo && c <= c_hi;
+              const float sc = sv[c] * p.inv;
+              const float s = in ? sc : 0.f;
+              a1[c & 1] += s;
+              a2[c & 1] = fmaf(s, s, a2[c & 1]);
+              if (in && sc > best) {   // columns ascend, so the first of equal maxima stays
+                best = sc;
+                best_v = vb + c;
+              }
+            }
+            s1 += static_cast<double>(a1[0] + a1[1]);
+            s2 += static_cast<double>(a2[0] + a2[1]);
+          }
+        } else if (ok) {
+          // lane l collects the counts of columns l and 32 + l from the
+          // column ballots, split between the warp's (at most two) query blocks
+          uint32_t n_lo[2] = {0u, 0u}, n_hi[2] = {0u, 0u};
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const bool kept = c >= c_lo && c <= c_hi && sv[c] * p.inv > thr_f;
+            const uint32_t bal = __ballot_sync(0xffffffffu, kept);
+            const uint32_t lo = __popc(bal & lanes_first), hi = __popc(bal & ~lanes_first);
+            if (lane == (c & 31)) {
+              n_lo[c >> 5] = lo;
+              n_hi[c >> 5] = hi;
             }
           }
-          s1 += static_cast<double>(a1[0] + a1[1]);
-          s2 += static_cast<double>(a2[0] + a2[1]);
-        }
-      } else if (ok) {
-        // lane l collects the counts of columns l and 32 + l from the
-        // column ballots, split between the warp's (at most two) query blocks
-        uint32_t n_lo[2] = {0u, 0u}, n_hi[2] = {0u, 0u};
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const bool kept = c >= c_lo && c <= c_hi && sv[c] * p.inv > thr_f;
-          const uint32_t bal = __ballot_sync(0xffffffffu, kept);
-          const uint32_t lo = __popc(bal & lanes_first), hi = __popc(bal & ~lanes_first);
-          if (lane == (c & 31)) {
-            n_lo[c >> 5] = lo;
-            n_hi[c >> 5] = hi;
+          for (int h = 0; h < 2; ++h) {
+            const int col = grp * 64 + h * 32 + lane;
+            if (n_lo[h] != 0u) atomicAdd(&ct[slot_first * C::kN + col], n_lo[h]);
+            if (n_hi[h] != 0u) atomicAdd(&ct[(slot_first + 1) * C::kN + col], n_hi[h]);
           }
         }
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int col = grp * 64 + h * 32 + lane;
-          if (n_lo[h] != 0u) atomicAdd(&ct[slot_first * C::kN + col], n_lo[h]);
-          if (n_hi[h] != 0u) atomicAdd(&ct[(slot_first + 1) * C::kN + col], n_hi[h]);
-        }
-      }
-      if (p.pass == 1) {
-        // the warpgroup's 64 columns of this tile are counted: add them to
-        // colcnt and clear them for tile jt + 2
-        asm volatile("bar.sync %0, 128;" ::"r"(1 + grp) : "memory");
-        const int tg = threadIdx.x - grp * 128;
-        const int v0 = v_lo + jt * C::kN;
-        for (int e = tg; e < kTokSlots * 64; e += 128) {
-          const int s_ = e / 64, col = grp * 64 + e % 64;
-          const uint32_t n = ct[s_ * C::kN + col];
-          if (n != 0u) {
-            atomicAdd(&p.colcnt[(static_cast<int64_t>(b) * g.nb + I0 + s_) * g.n + j * nt + v0 + col], n);
-            ct[s_ * C::kN + col] = 0u;
+        if (p.pass == 1) {
+          // the warpgroup's 64 columns of this tile are counted: add them to
+          // colcnt and clear them for tile gt + 2
+          asm volatile("bar.sync %0, 128;" ::"r"(1 + grp) : "memory");
+          const int tg = threadIdx.x - grp * 128;
+          const int v0 = x.v_lo + jt * C::kN;
+          for (int e = tg; e < kTokSlots * 64; e += 128) {
+            const int s_ = e / 64, col = grp * 64 + e % 64;
+            const uint32_t n = ct[s_ * C::kN + col];
+            if (n != 0u) {
+              if (ok)
+                atomicAdd(&p.colcnt[(static_cast<int64_t>(x.b) * g.nb + I0 + s_) * g.n + x.j * nt + v0 + col], n);
+              ct[s_ * C::kN + col] = 0u;
+            }
           }
         }
       }
-    }
-    if (p.pass == 0) {
-      unsigned long long key = 0ull;
-      if (best_v >= 0)
-        key = (static_cast<unsigned long long>(tok_order_key(best)) << 32) |
-              (0xFFFFFFFFull - static_cast<unsigned long long>(u * nt + best_v));
+      if (p.pass == 0) {
+        // the unit's sums and first maximum: warp, then the 8 epilogue warps
+        unsigned long long key = 0ull;
+        if (best_v >= 0)
+          key = (static_cast<unsigned long long>(tok_order_key(best)) << 32) |
+                (0xFFFFFFFFull - static_cast<unsigned long long>(u * nt + best_v));
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        s1 += __shfl_xor_sync(0xffffffffu, s1, off);
-        s2 += __shfl_xor_sync(0xffffffffu, s2, off);
-        const unsigned long long o = __shfl_xor_sync(0xffffffffu, key, off);
-        key = o > key ? o : key;
+        for (int off = 16; off > 0; off >>= 1) {
+          s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+          s2 += __shfl_xor_sync(0xffffffffu, s2, off);
+          const unsigned long long o = __shfl_xor_sync(0xffffffffu, key, off);
+          key = o > key ? o : key;
+        }
+        const int par = ul & 1;
+        if (lane == 0) {
+          red_d[par * 16 + warp] = s1;
+          red_d[par * 16 + 8 + warp] = s2;
+          red_b[par * 8 + warp] = key;
+        }
+        asm volatile("bar.sync 3, 256;" ::: "memory");
+        if (threadIdx.x == 0 && ok) {
+          double a1 = 0.0, a2 = 0.0;
+          unsigned long long bb = 0ull;
+          for (int q = 0; q < 8; ++q) {
+            a1 += red_d[par * 16 + q];
+            a2 += red_d[par * 16 + 8 + q];
+            bb = red_b[par * 8 + q] > bb ? red_b[par * 8 + q] : bb;
+          }
+          double* st = p.stats + (static_cast<int64_t>(x.b) * F * F + x.pi) * 2;
+          atomicAdd(st, a1);
+          atomicAdd(st + 1, a2);
+          atomicMax(&p.best[static_cast<int64_t>(x.b) * F * F + x.pi], bb);
+        }
       }
-      if (lane == 0) {
-        red_d[warp] = s1;
-        red_d[8 + warp] = s2;
-        red_b[warp] = key;
-      }
+      ++ul;
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (p.pass == 0 && threadIdx.x == 0 && !*abort_flag) {
-    double a1 = 0.0, a2 = 0.0;
-    unsigned long long bb = 0ull;
-    for (int x = 0; x < 8; ++x) {
-      a1 += red_d[x];
-      a2 += red_d[8 + x];
-      bb = red_b[x] > bb ? red_b[x] : bb;
-    }
-    double* st = p.stats + (static_cast<int64_t>(b) * F * F + pi) * 2;
-    atomicAdd(st, a1);
-    atomicAdd(st + 1, a2);
-    atomicMax(&p.best[static_cast<int64_t>(b) * F * F + pi], bb);
-  }
   if (warp == 9) tmem_dealloc(taddr, C::kTmemCols);
 }
 
