@@ -560,6 +560,8 @@ int dynrad_build_sampled_mask(const dynrad_geom* geom, double rho1, double rho2,
   if (g.block != 32 && g.block != 64 && g.block != 128) return DYNRAD_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(replicas) * g.nb + 1 > INT32_MAX) return DYNRAD_ERR_UNSUPPORTED;
   if ((static_cast<int64_t>(g.nt) + kSampleRowsPerCta - 1) / kSampleRowsPerCta > 65535) return DYNRAD_ERR_UNSUPPORTED;
+  // the marking keeps a frame table and one flag per candidate in default shared memory
+  if (static_cast<size_t>(g.frames) * 5 + static_cast<size_t>(g.nb) + 16 > 48 * 1024) return DYNRAD_ERR_UNSUPPORTED;
   const SampleWorkspace w = sample_layout(g.frames, g.nb, cand_nnz);
   if (workspace_bytes < w.total) return DYNRAD_ERR_CAPACITY;
   cudaStream_t st = as_stream(stream);
@@ -592,7 +594,7 @@ int dynrad_build_sampled_mask(const dynrad_geom* geom, double rho1, double rho2,
     sample_pick_kernel<<<fp, kSampleThreads, 0, st>>>(sp);
     if ((rc = launch_status()) != DYNRAD_OK) return rc;
   }
-  const size_t msmem = static_cast<size_t>(g.frames) * 5 + 16;
+  const size_t msmem = static_cast<size_t>(g.frames) * 5 + static_cast<size_t>(g.nb) + 16;
   if (g.block == 32) sample_mark_kernel<32><<<g.nb, kSampleThreads, msmem, st>>>(sp);
   else if (g.block == 64) sample_mark_kernel<64><<<g.nb, kSampleThreads, msmem, st>>>(sp);
   else sample_mark_kernel<128><<<g.nb, kSampleThreads, msmem, st>>>(sp);

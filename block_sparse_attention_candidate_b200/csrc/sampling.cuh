@@ -17,8 +17,8 @@
 //   sample_hist_kernel    one radix pass (11-bit digit, 6 passes for 64 bits):
 //                         histogram of the keys that share the digits found.
 //   sample_pick_kernel    per frame pair: the digit holding the k-th key.
-//   sample_mark_kernel    per query block: token-level sampled links of each
-//                         candidate block, (theta_c, theta_m) aggregation.
+//   sample_mark_kernel    per query block, one warp per candidate block: its
+//                         token-level sampled links, (theta_c, theta_m).
 //   replicate_csr_kernel  copies the head-shared CSR for every (batch, head).
 #pragma once
 
@@ -214,58 +214,72 @@ __global__ void __launch_bounds__(kSampleThreads) sample_pick_kernel(SampleParam
 // Per query block I: for each candidate block J (ascending), J is kept if it
 // is in F_I or if, over the sampled token links of (I, J), more than
 // theta_m * n_J of J's columns are active (a column is active when more than
-// theta_c * n_I of I's tokens link to it).
+// theta_c * n_I of I's tokens link to it).  One warp per candidate (eight at a
+// time): lanes take J's columns and walk I's tokens; then warp 0 writes the
+// kept candidates in list order.
 template <int BS>
 __global__ void __launch_bounds__(kSampleThreads) sample_mark_kernel(SampleParams p) {
   extern __shared__ __align__(16) uint8_t sm_raw[];
   const GeomDev& g = p.g;
   int* wt = reinterpret_cast<int*>(sm_raw);                    // [F]
   uint8_t* rt = reinterpret_cast<uint8_t*>(wt + g.frames);     // [F]
-  __shared__ uint32_t colcnt[BS];
-  __shared__ int n_kept;
+  uint8_t* keep = rt + g.frames;                               // [nb] per list position
+  constexpr int kColsPerLane = (BS + 31) / 32;
   const int I = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   build_frame_tables(g, wt, rt);
-  if (threadIdx.x == 0) n_kept = 0;
   __syncthreads();
   const int q0 = I * BS, q1 = min(q0 + BS, g.n);
   const int nI = q1 - q0;
-  const int c_beg = p.cand_row_ptr[I], c_end = p.cand_row_ptr[I + 1];
-  const int flo = p.forced_lo[I], fhi = p.forced_hi[I];
-  constexpr int kQSplit = kSampleThreads / BS;   // threads per column
-  const int col = threadIdx.x % BS, qs = threadIdx.x / BS;
-  for (int c = c_beg; c < c_end; ++c) {
-    const int J = p.cand_col[c];
-    bool keep = J >= flo && J <= fhi;
-    if (!keep) {
-      const int k0 = J * BS, k1 = min(k0 + BS, g.n);
-      const int nJ = k1 - k0;
-      if (threadIdx.x < BS) colcnt[threadIdx.x] = 0u;
-      __syncthreads();
-      const int k = k0 + col;
-      if (k < k1) {
-        const int j = k / g.nt, v = k % g.nt;
-        uint32_t cnt = 0;
-        for (int q = q0 + qs; q < q1; q += kQSplit) {
-          const int i = q / g.nt, u = q % g.nt;
-          const int t = i > j ? i - j : j - i;
-          const int d = u > v ? u - v : v - u;
-          if (!rt[t] || d > wt[t]) continue;   // not in P(i, j)
-          if (t >= 2 &&
-              sample_key(p.seed, g.frames, g.nt, i, j, u, v) > p.thresholds[static_cast<int64_t>(i) * g.frames + j])
-            continue;                          // not sampled
-          ++cnt;
-        }
-        if (cnt) atomicAdd(&colcnt[col], cnt);
-      }
-      __syncthreads();
-      const bool active = threadIdx.x < nJ && static_cast<double>(colcnt[threadIdx.x]) > g.theta_c * nI;
-      const int n_active = __syncthreads_count(active);
-      keep = static_cast<double>(n_active) > g.theta_m * nJ;
-    }
-    if (keep && threadIdx.x == 0) p.kept_tmp[c_beg + n_kept++] = J;
-    __syncthreads();
+  const int c_beg = p.cand_row_ptr[I];
+  int nc = p.cand_row_ptr[I + 1] - c_beg;
+  if (nc > g.nb || nc < 0) {   // not a valid candidate row
+    if (threadIdx.x == 0) record_error(DYNRAD_ERR_CAPACITY);
+    nc = nc < 0 ? 0 : g.nb;
   }
-  if (threadIdx.x == 0) p.counts[I] = n_kept;
+  const int flo = p.forced_lo[I], fhi = p.forced_hi[I];
+  const double need_links = g.theta_c * nI;
+  for (int c = warp; c < nc; c += kSampleThreads / 32) {
+    const int J = p.cand_col[c_beg + c];
+    bool kp = J >= flo && J <= fhi;
+    if (!kp) {
+      const int k0 = J * BS, k1 = min(k0 + BS, g.n), nJ = k1 - k0;
+      int n_active = 0;
+#pragma unroll
+      for (int x = 0; x < kColsPerLane; ++x) {
+        const int k = k0 + lane + 32 * x;
+        uint32_t cnt = 0;
+        if (k < k1) {
+          const int j = k / g.nt, v = k % g.nt;
+          for (int q = q0; q < q1; ++q) {
+            const int i = q / g.nt, u = q % g.nt;
+            const int t = i > j ? i - j : j - i;
+            const int d = u > v ? u - v : v - u;
+            if (!rt[t] || d > wt[t]) continue;   // not in P(i, j)
+            if (t >= 2 &&
+                sample_key(p.seed, g.frames, g.nt, i, j, u, v) > p.thresholds[static_cast<int64_t>(i) * g.frames + j])
+              continue;                          // not sampled
+            ++cnt;
+          }
+        }
+        n_active += __popc(__ballot_sync(0xffffffffu, k < k1 && static_cast<double>(cnt) > need_links));
+      }
+      kp = static_cast<double>(n_active) > g.theta_m * nJ;
+    }
+    if (lane == 0) keep[c] = kp ? 1 : 0;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int n_kept = 0;
+    for (int c0 = 0; c0 < nc; c0 += 32) {
+      const int c = c0 + lane;
+      const bool k_ = c < nc && keep[c] != 0;
+      const unsigned bal = __ballot_sync(0xffffffffu, k_);
+      if (k_) p.kept_tmp[c_beg + n_kept + __popc(bal & ((1u << lane) - 1u))] = p.cand_col[c_beg + c];
+      n_kept += __popc(bal);
+    }
+    if (lane == 0) p.counts[I] = n_kept;
+  }
 }
 
 // Copies replica 0 of the CSR (rows [0, nb), entries [0, nnz)) to replicas
