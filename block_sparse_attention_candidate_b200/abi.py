@@ -42,6 +42,7 @@ EXPORTED = (
     "dynrad_host_path_workspace_bytes",
     "dynrad_host_path",
     "dynrad_sampled_mask_workspace_bytes",
+    "dynrad_sampled_mask_workspace_min_bytes",
     "dynrad_build_sampled_mask",
     "dynrad_token_mask_workspace_bytes",
     "dynrad_build_token_mask",
@@ -142,6 +143,8 @@ def lib() -> ctypes.CDLL:
                                        _I32, ctypes.c_float, _VP, _SZ, _VP]
         L.dynrad_sampled_mask_workspace_bytes.restype = _SZ
         L.dynrad_sampled_mask_workspace_bytes.argtypes = [_GP, _I64]
+        L.dynrad_sampled_mask_workspace_min_bytes.restype = _SZ
+        L.dynrad_sampled_mask_workspace_min_bytes.argtypes = [_GP, _I64]
         L.dynrad_build_sampled_mask.restype = ctypes.c_int
         L.dynrad_build_sampled_mask.argtypes = [_GP, ctypes.c_double, ctypes.c_double, ctypes.c_uint64, _VP, _VP, _I64,
                                                 _VP, _VP, _I32, _VP, _VP, _I64, _VP, _VP, _SZ, _VP]
@@ -420,17 +423,23 @@ def dynrad_host_path(q_host, k_host, v_host, runs, chunk_bh=4, scale=0.0, worksp
     return ws
 
 
-def dynrad_build_sampled_mask(geom, cand, rho1, rho2, seed, replicas=1, thresholds=False, stream=None):
+def dynrad_build_sampled_mask(geom, cand, rho1, rho2, seed, replicas=1, thresholds=False, stream=None,
+                              workspace_bytes=None):
     """Paper-exact static-ratio mask (Eq. 8, seeded token-pair sampling), the
     same for every head, written ``replicas`` times.  Returns (row_ptr int32
     [replicas*Nb+1], col_idx int32 with capacity replicas*cand_nnz, thresholds
-    int64 [F*F] holding the uint64 T(i, j) bits, or None)."""
+    int64 [F*F] holding the uint64 T(i, j) bits, or None).  ``workspace_bytes``
+    (default: the full size) may be anything from
+    dynrad_sampled_mask_workspace_min_bytes up; a smaller pool only slows the
+    build."""
     L = lib()
     cg = make_geom(geom)
     device = cand["row_ptr"].device
     ws_bytes = int(L.dynrad_sampled_mask_workspace_bytes(ctypes.byref(cg), cand["nnz"]))
     if ws_bytes == 0:
         raise DynradError(DYNRAD_ERR_INVALID_ARG, "dynrad_sampled_mask_workspace_bytes")
+    if workspace_bytes is not None:
+        ws_bytes = int(workspace_bytes)
     ws = torch.empty(ws_bytes + 256, dtype=torch.uint8, device=device)
     off = (-ws.data_ptr()) % 256
     nb = cand["nb"]

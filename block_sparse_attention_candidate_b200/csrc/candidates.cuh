@@ -15,6 +15,8 @@
 // double arithmetic.
 #pragma once
 
+#include <cmath>
+
 #include "common.cuh"
 
 namespace dynrad {
@@ -25,29 +27,61 @@ struct GeomDev {
   double gamma, lambda, theta_c, theta_m, eps;
 };
 
+// Correctly rounded double steps.  On the device the explicit intrinsics keep
+// nvcc from contracting a multiply-add into an FMA; on the host (x86-64 SSE2
+// double, no FMA contraction) the plain operators round the same way.  The host
+// forms only size workspaces.
+__host__ __device__ __forceinline__ double geo_mul(double a, double b) {
+#ifdef __CUDA_ARCH__
+  return __dmul_rn(a, b);
+#else
+  return a * b;
+#endif
+}
+__host__ __device__ __forceinline__ double geo_add(double a, double b) {
+#ifdef __CUDA_ARCH__
+  return __dadd_rn(a, b);
+#else
+  return a + b;
+#endif
+}
+__host__ __device__ __forceinline__ double geo_div(double a, double b) {
+#ifdef __CUDA_ARCH__
+  return __ddiv_rn(a, b);
+#else
+  return a / b;
+#endif
+}
+
 // B(t) of Eq. 1 for t >= 1: floor(log2 t) + 1 = bit length of t.
-__device__ __forceinline__ int log_group(int t) { return 32 - __clz(t); }
+__host__ __device__ __forceinline__ int log_group(int t) {
+#ifdef __CUDA_ARCH__
+  return 32 - __clz(t);
+#else
+  return 32 - __builtin_clz(static_cast<unsigned>(t));
+#endif
+}
 
 // L0 / 2^B(t), exact in double.
-__device__ __forceinline__ double span_over_group(int64_t l0, int t) {
+__host__ __device__ __forceinline__ double span_over_group(int64_t l0, int t) {
   return ldexp(static_cast<double>(l0), -log_group(t));
 }
 
 // w(t) of Eq. 3, clamped to N_t (every |u - v| is below N_t).
-__device__ __forceinline__ int window_width(const GeomDev& g, int t) {
+__host__ __device__ __forceinline__ int window_width(const GeomDev& g, int t) {
   if (t <= 1) return g.nt;
-  const double L = __dmul_rn(span_over_group(g.l0, t), g.gamma);  // Eq. 2
-  const double r = floor(__dadd_rn(L, 0.5));                      // round half up
+  const double L = geo_mul(span_over_group(g.l0, t), g.gamma);  // Eq. 2
+  const double r = floor(geo_add(L, 0.5));                      // round half up
   long long w = r > 4.0e18 ? (long long)4e18 : (long long)r;
   if (w < g.block) w = g.block;
   return w > g.nt ? g.nt : static_cast<int>(w);
 }
 
 // Eq. 6: t mod sf(t) == 0, sf(t) = max(1, floor(B_s / (L_split(t) + eps))).
-__device__ __forceinline__ bool pair_retained(const GeomDev& g, int t) {
+__host__ __device__ __forceinline__ bool pair_retained(const GeomDev& g, int t) {
   if (t == 0) return true;
-  const double ls = __dmul_rn(span_over_group(g.l0, t), g.lambda);  // Eq. 4
-  const double qf = floor(__ddiv_rn(static_cast<double>(g.block), __dadd_rn(ls, g.eps)));
+  const double ls = geo_mul(span_over_group(g.l0, t), g.lambda);  // Eq. 4
+  const double qf = floor(geo_div(static_cast<double>(g.block), geo_add(ls, g.eps)));
   if (qf > static_cast<double>(t)) return false;  // sf > t >= 1: t mod sf = t != 0
   long long sf = static_cast<long long>(qf);
   if (sf < 1) sf = 1;

@@ -519,19 +519,36 @@ int dynrad_select_blocks(const void* q, const void* k, int32_t B, int32_t H, int
 namespace {
 
 struct SampleWorkspace {
-  size_t pairs, hist, thresholds, kept, partial, total;
+  size_t pairs, counters, thresholds, kept, partial, pool, total;
 };
 
-SampleWorkspace sample_layout(int64_t frames, int64_t nb, int64_t cand_nnz) {
+// Pool slots for every sampled frame pair at its largest window (q = 1/2):
+// sum over distances t >= 2 kept by the split rule of 2 (F - t) ordered pairs.
+uint64_t sample_pool_keys(const GeomDev& g) {
+  uint64_t total = 0;
+  const int64_t nt = g.nt;
+  for (int t = 2; t < g.frames; ++t) {
+    if (!pair_retained(g, t)) continue;
+    const int64_t w = window_width(g, t), wc = w < nt - 1 ? w : nt - 1;
+    const double n = static_cast<double>(nt * (2 * wc + 1) - wc * (wc + 1));
+    if (n <= 0.0) continue;
+    const double e = kSampleWindowDevs * sqrt(n) + 2.0 * kSampleWindowPad;
+    total += 2ull * static_cast<uint64_t>(g.frames - t) * (sample_pool_slots(n, e) + 2ull);
+  }
+  return total;
+}
+
+SampleWorkspace sample_layout(const GeomDev& g, int64_t cand_nnz, bool with_pool) {
   SampleWorkspace w;
-  const int64_t fp = frames * frames;
-  const int64_t tiles = (nb + 1 + kScanTile - 1) / kScanTile;
+  const int64_t fp = static_cast<int64_t>(g.frames) * g.frames;
+  const int64_t tiles = (g.nb + 1 + kScanTile - 1) / kScanTile;
   w.pairs = 0;
-  w.hist = align256(w.pairs + static_cast<size_t>(fp) * sizeof(SamplePair));
-  w.thresholds = align256(w.hist + static_cast<size_t>(fp) * kSampleBins * 4);
+  w.counters = align256(w.pairs + static_cast<size_t>(fp) * sizeof(SamplePair));
+  w.thresholds = align256(w.counters + static_cast<size_t>(2 * fp + 1) * 8);
   w.kept = align256(w.thresholds + static_cast<size_t>(fp) * 8);
   w.partial = align256(w.kept + static_cast<size_t>(cand_nnz) * 4);
-  w.total = align256(w.partial + static_cast<size_t>(tiles) * 8);
+  w.pool = align256(w.partial + static_cast<size_t>(tiles) * 8);
+  w.total = with_pool ? align256(w.pool + static_cast<size_t>(sample_pool_keys(g)) * 8) : w.pool;
   return w;
 }
 
@@ -540,7 +557,13 @@ SampleWorkspace sample_layout(int64_t frames, int64_t nb, int64_t cand_nnz) {
 size_t dynrad_sampled_mask_workspace_bytes(const dynrad_geom* geom, int64_t cand_nnz) {
   GeomDev g;
   if (check_geom(geom, &g) != DYNRAD_OK || cand_nnz < 1) return 0;
-  return sample_layout(g.frames, g.nb, cand_nnz).total;
+  return sample_layout(g, cand_nnz, true).total;
+}
+
+size_t dynrad_sampled_mask_workspace_min_bytes(const dynrad_geom* geom, int64_t cand_nnz) {
+  GeomDev g;
+  if (check_geom(geom, &g) != DYNRAD_OK || cand_nnz < 1) return 0;
+  return sample_layout(g, cand_nnz, false).total;
 }
 
 int dynrad_build_sampled_mask(const dynrad_geom* geom, double rho1, double rho2, uint64_t seed,
@@ -562,17 +585,22 @@ int dynrad_build_sampled_mask(const dynrad_geom* geom, double rho1, double rho2,
   if ((static_cast<int64_t>(g.nt) + kSampleRowsPerCta - 1) / kSampleRowsPerCta > 65535) return DYNRAD_ERR_UNSUPPORTED;
   // the marking keeps a frame table and one flag per candidate in default shared memory
   if (static_cast<size_t>(g.frames) * 5 + static_cast<size_t>(g.nb) + 16 > 48 * 1024) return DYNRAD_ERR_UNSUPPORTED;
-  const SampleWorkspace w = sample_layout(g.frames, g.nb, cand_nnz);
+  const SampleWorkspace w = sample_layout(g, cand_nnz, false);
   if (workspace_bytes < w.total) return DYNRAD_ERR_CAPACITY;
   cudaStream_t st = as_stream(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int fp = g.frames * g.frames;
   SampleParams sp;
   sp.g = g;
   sp.rho1 = rho1;
   sp.rho2 = rho2;
   sp.seed = seed;
   sp.pairs = reinterpret_cast<SamplePair*>(ws + w.pairs);
-  sp.hist = reinterpret_cast<uint32_t*>(ws + w.hist);
+  sp.below = reinterpret_cast<unsigned long long*>(ws + w.counters);
+  sp.inwin = sp.below + fp;
+  sp.pool_used = sp.inwin + fp;
+  sp.pool = reinterpret_cast<uint64_t*>(ws + w.pool);
+  sp.pool_cap = (workspace_bytes - w.pool) / 8;   // whatever the caller gave beyond the fixed part
   sp.thresholds = reinterpret_cast<uint64_t*>(ws + w.thresholds);
   sp.cand_row_ptr = cand_row_ptr;
   sp.cand_col = cand_col;
@@ -580,20 +608,14 @@ int dynrad_build_sampled_mask(const dynrad_geom* geom, double rho1, double rho2,
   sp.forced_hi = forced_hi;
   sp.counts = row_ptr;
   sp.kept_tmp = reinterpret_cast<int32_t*>(ws + w.kept);
-  sp.pass = 0;
-  const int fp = g.frames * g.frames;
+  if (cudaMemsetAsync(sp.below, 0, static_cast<size_t>(2 * fp + 1) * 8, st) != cudaSuccess) return DYNRAD_ERR_CUDA;
   sample_setup_kernel<<<(fp + 255) / 256, 256, 0, st>>>(sp);
   if ((rc = launch_status()) != DYNRAD_OK) return rc;
-  if (cudaMemsetAsync(sp.hist, 0, static_cast<size_t>(fp) * kSampleBins * 4, st) != cudaSuccess)
-    return DYNRAD_ERR_CUDA;
-  const dim3 hgrid(fp, (g.nt + kSampleRowsPerCta - 1) / kSampleRowsPerCta);
-  for (int pass = 0; pass < kSamplePasses; ++pass) {
-    sp.pass = pass;
-    sample_hist_kernel<<<hgrid, kSampleThreads, 0, st>>>(sp);
-    if ((rc = launch_status()) != DYNRAD_OK) return rc;
-    sample_pick_kernel<<<fp, kSampleThreads, 0, st>>>(sp);
-    if ((rc = launch_status()) != DYNRAD_OK) return rc;
-  }
+  const dim3 cgrid(fp, (g.nt + kSampleRowsPerCta - 1) / kSampleRowsPerCta);
+  sample_collect_kernel<<<cgrid, kSampleThreads, 0, st>>>(sp);
+  if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  sample_select_kernel<<<fp, kSampleThreads, 0, st>>>(sp);
+  if ((rc = launch_status()) != DYNRAD_OK) return rc;
   const size_t msmem = static_cast<size_t>(g.frames) * 5 + static_cast<size_t>(g.nb) + 16;
   if (g.block == 32) sample_mark_kernel<32><<<g.nb, kSampleThreads, msmem, st>>>(sp);
   else if (g.block == 64) sample_mark_kernel<64><<<g.nb, kSampleThreads, msmem, st>>>(sp);

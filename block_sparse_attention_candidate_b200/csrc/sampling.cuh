@@ -12,14 +12,28 @@
 // never tie; the sample is the k pairs with the smallest keys, i.e. every pair
 // whose key is <= T(i, j), the k-th smallest key.
 //
+// Finding T(i, j) exactly in one pass over the keys.  The keys of a frame pair
+// are spread uniformly over [0, 2^64), so the k-th smallest lies near
+// (k - 1/2) / |P| * 2^64, within a few sqrt(q (1 - q) / |P|) * 2^64 (q = k / |P|,
+// the spread of a uniform order statistic).  One pass counts the keys below a
+// window [lo, hi] around that point (7 such deviations plus 64 keys' worth on
+// each side) and copies the keys inside it to a per-pair pool; if the counts
+// show that the window holds the k-th key, a radix select over the few
+// thousand pooled keys gives T.  Otherwise (never seen with real keys, but
+// possible for a pair whose pool reservation did not fit the workspace) the
+// select CTA recomputes all of the pair's keys in each radix pass.  Either way
+// T is the exact k-th smallest key.
+//
 // Kernels:
-//   sample_setup_kernel   per frame pair: window, |P| (closed form), rho, k.
-//   sample_hist_kernel    one radix pass (11-bit digit, 6 passes for 64 bits):
-//                         histogram of the keys that share the digits found.
-//   sample_pick_kernel    per frame pair: the digit holding the k-th key.
-//   sample_mark_kernel    per query block, one warp per candidate block: its
-//                         token-level sampled links, (theta_c, theta_m).
-//   replicate_csr_kernel  copies the head-shared CSR for every (batch, head).
+//   sample_setup_kernel    per frame pair: window, |P| (closed form), rho, k,
+//                          the key window and its pool reservation.
+//   sample_collect_kernel  one pass over every key: counts below the window,
+//                          pools the keys inside it.
+//   sample_select_kernel   per frame pair: 11-bit radix select of the k-th key
+//                          over the pooled keys (or over all keys).
+//   sample_mark_kernel     per query block, one warp per candidate block: its
+//                          token-level sampled links, (theta_c, theta_m).
+//   replicate_csr_kernel   copies the head-shared CSR for every (batch, head).
 #pragma once
 
 #include "candidates.cuh"
@@ -31,19 +45,33 @@ constexpr int kSampleDigitBits = 11;
 constexpr int kSampleBins = 1 << kSampleDigitBits;   // 2048
 constexpr int kSamplePasses = 6;                     // 5 x 11 + 9 bits
 constexpr int kSampleThreads = 256;
-constexpr int kSampleRowsPerCta = 32;                // u rows of a frame pair per histogram CTA
+constexpr int kSampleRowsPerCta = 64;                // u rows of a frame pair per collect CTA
+constexpr uint64_t kSplitMixGamma = 0x9E3779B97F4A7C15ull;
+constexpr double kSampleWindowDevs = 7.0;            // window half-width in order-statistic deviations
+constexpr double kSampleWindowPad = 64.0;            // plus this many keys' worth on each side
 
 __host__ __device__ constexpr int sample_shift(int pass) { return pass < 5 ? 53 - 11 * pass : 0; }
 __host__ __device__ constexpr int sample_width(int pass) { return pass < 5 ? 11 : 9; }
 
+// Pool slots reserved for a pair with |P| = n: ceil(e + 8 sqrt(e) + 64), at
+// most n, e the expected number of keys in the window.  The host sizes the
+// pool with the same function at e's largest value (q = 1/2).
+__host__ __device__ inline uint64_t sample_pool_slots(double n, double expect) {
+  double c = ceil(expect + 8.0 * sqrt(expect) + 64.0);
+  if (c > n) c = n;
+  if (c > 2147483647.0) c = 2147483647.0;
+  return static_cast<uint64_t>(c);
+}
+
 struct SamplePair {
   uint64_t n;       // |P(i, j)|
   uint64_t k;       // sample size
-  uint64_t prefix;  // key digits found so far (then T)
-  uint64_t rank;    // 1-based rank of the k-th key among keys sharing the prefix
+  uint64_t lo, hi;  // key window expected to hold the k-th smallest key
+  uint64_t off;     // first pool slot
+  uint32_t cap;     // pool slots reserved (0: none; the select recomputes every key)
   int32_t w;        // window half-width (clamped to N_t)
   int32_t active;   // sampled by key (t >= 2, retained, |P| > 0)
-  int32_t pad[2];
+  int32_t pad;
 };
 
 struct SampleParams {
@@ -51,7 +79,11 @@ struct SampleParams {
   double rho1, rho2;
   uint64_t seed;
   SamplePair* pairs;        // [F * F]
-  uint32_t* hist;           // [F * F][kSampleBins]
+  unsigned long long* below;   // [F * F] keys below lo (zeroed before setup)
+  unsigned long long* inwin;   // [F * F] keys in [lo, hi] (zeroed before setup)
+  unsigned long long* pool_used;  // slots handed out (zeroed before setup)
+  uint64_t* pool;           // [pool_cap] pooled window keys
+  uint64_t pool_cap;
   uint64_t* thresholds;     // [F * F] T(i, j); UINT64_MAX where every pair of P is kept
   const int32_t* cand_row_ptr;
   const int32_t* cand_col;
@@ -59,7 +91,6 @@ struct SampleParams {
   const int32_t* forced_hi;
   int32_t* counts;          // [nb] kept per row
   int32_t* kept_tmp;        // [cand_nnz] kept lists at the candidate offsets
-  int pass;
 };
 
 __device__ __forceinline__ uint64_t splitmix64_mix(uint64_t z) {
@@ -68,9 +99,16 @@ __device__ __forceinline__ uint64_t splitmix64_mix(uint64_t z) {
   return z ^ (z >> 31);
 }
 
-__device__ __forceinline__ uint64_t sample_key(uint64_t seed, int frames, int nt, int i, int j, int u, int v) {
+// The generator state before mixing for counter c: seed + (c + 1) * gamma
+// (mod 2^64).  Consecutive v add gamma, consecutive u add N_t * gamma, so the
+// scans below step the state instead of recomputing it.
+__device__ __forceinline__ uint64_t sample_state(uint64_t seed, int frames, int nt, int i, int j, int u, int v) {
   const uint64_t c = ((static_cast<uint64_t>(i) * frames + j) * nt + u) * nt + v;
-  return splitmix64_mix(seed + (c + 1ull) * 0x9E3779B97F4A7C15ull);
+  return seed + (c + 1ull) * kSplitMixGamma;
+}
+
+__device__ __forceinline__ uint64_t sample_key(uint64_t seed, int frames, int nt, int i, int j, int u, int v) {
+  return splitmix64_mix(sample_state(seed, frames, nt, i, j, u, v));
 }
 
 __global__ void sample_setup_kernel(SampleParams p) {
@@ -97,118 +135,169 @@ __global__ void sample_setup_kernel(SampleParams p) {
     s.k = k > s.n ? s.n : k;
   }
   s.active = (t >= 2 && s.n > 0) ? 1 : 0;
-  s.prefix = 0ull;
-  s.rank = s.k;
-  s.pad[0] = s.pad[1] = 0;
+  s.lo = 0ull;
+  s.hi = ~0ull;
+  s.off = 0ull;
+  s.cap = 0u;
+  s.pad = 0;
+  if (s.active) {
+    // Any window is correct (the select checks the counts); this one holds
+    // the k-th key unless it sits more than 7 deviations from its mean.
+    const double n = static_cast<double>(s.n), q = static_cast<double>(s.k) / n;
+    const double half = kSampleWindowDevs * sqrt(q * (1.0 - q) / n) + kSampleWindowPad / n;
+    const double mid = (static_cast<double>(s.k) - 0.5) / n;
+    const double lo_f = mid - half, hi_f = mid + half;
+    const double two64 = 18446744073709551616.0;
+    if (lo_f > 0.0) s.lo = static_cast<uint64_t>(lo_f * two64);   // lo_f < mid < 1
+    if (hi_f < 1.0 - 0x1p-40) s.hi = static_cast<uint64_t>(hi_f * two64);
+    const double span = fmin(hi_f, 1.0) - fmax(lo_f, 0.0);
+    const uint64_t cap = sample_pool_slots(n, span * n);
+    const unsigned long long off = atomicAdd(p.pool_used, static_cast<unsigned long long>(cap));
+    if (off + cap <= p.pool_cap) {
+      s.off = off;
+      s.cap = static_cast<uint32_t>(cap);
+    }
+  }
   p.pairs[idx] = s;
   p.thresholds[idx] = ~0ull;
 }
 
-// Histogram of one 11-bit digit over the keys of frame pair blockIdx.x, rows
-// u in [blockIdx.y * 32, +32), that agree with the digits found so far.
-__global__ void __launch_bounds__(kSampleThreads) sample_hist_kernel(SampleParams p) {
+// One pass over the keys of frame pair blockIdx.x, rows u in
+// [blockIdx.y * 64, +64), one warp per row (lanes over v): counts the keys
+// below the pair's window and appends the keys inside it to the pair's pool
+// slots (in any order).
+__global__ void __launch_bounds__(kSampleThreads) sample_collect_kernel(SampleParams p) {
+  __shared__ unsigned long long wsum[kSampleThreads / 32];
+  const int F = p.g.frames, nt = p.g.nt;
+  const int pi = blockIdx.x;
+  const SamplePair s = p.pairs[pi];
+  if (!s.active || s.cap == 0u) return;   // no pool: the select pass reads every key itself
+  const int u0 = blockIdx.y * kSampleRowsPerCta;
+  if (u0 >= nt) return;
+  const int u1 = min(u0 + kSampleRowsPerCta, nt);
+  const int i = pi / F, j = pi % F;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint64_t step = 32ull * kSplitMixGamma;
+  uint32_t below = 0;
+  for (int u = u0 + warp; u < u1; u += kSampleThreads / 32) {   // warp-uniform
+    const int va = max(u - s.w, 0), vb = min(u + s.w, nt - 1);
+    uint64_t z = sample_state(p.seed, F, nt, i, j, u, va + lane);
+    for (int v0 = va; v0 <= vb; v0 += 32, z += step) {          // warp-uniform
+      const bool valid = v0 + lane <= vb;
+      const uint64_t key = splitmix64_mix(z);
+      below += (valid && key < s.lo) ? 1u : 0u;
+      const bool in_win = valid && key >= s.lo && key <= s.hi;
+      const unsigned m = __ballot_sync(0xffffffffu, in_win);
+      if (m != 0u) {
+        const int leader = __ffs(m) - 1;
+        unsigned long long base = 0;
+        if (lane == leader) base = atomicAdd(&p.inwin[pi], static_cast<unsigned long long>(__popc(m)));
+        base = __shfl_sync(0xffffffffu, base, leader);
+        if (in_win) {
+          const unsigned long long pos = base + __popc(m & ((1u << lane) - 1u));
+          if (pos < s.cap) p.pool[s.off + pos] = key;   // beyond cap: the select falls back
+        }
+      }
+    }
+  }
+  unsigned long long bsum = below;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) bsum += __shfl_xor_sync(0xffffffffu, bsum, o);
+  if (lane == 0) wsum[warp] = bsum;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long sum = 0;
+    for (int x = 0; x < kSampleThreads / 32; ++x) sum += wsum[x];
+    if (sum != 0ull) atomicAdd(&p.below[pi], sum);
+  }
+}
+
+// Per frame pair: T(i, j), the k-th smallest key, by six 11-bit radix passes
+// (top digit first) over the pooled window keys when the counts show that the
+// window holds it, else over all of the pair's keys, recomputed each pass.
+__global__ void __launch_bounds__(kSampleThreads) sample_select_kernel(SampleParams p) {
+  constexpr int kPer = kSampleBins / kSampleThreads;   // 8 bins per thread
   __shared__ uint32_t h[kSampleBins];
-  __shared__ int32_t rstart[kSampleRowsPerCta + 1];
+  __shared__ unsigned long long wsum[kSampleThreads / 32];
+  __shared__ int found_bin;
+  __shared__ unsigned long long found_below;
   const int F = p.g.frames, nt = p.g.nt;
   const int pi = blockIdx.x;
   const SamplePair s = p.pairs[pi];
   if (!s.active) return;
-  const int u0 = blockIdx.y * kSampleRowsPerCta;
-  if (u0 >= nt) return;
-  const int rows = min(kSampleRowsPerCta, nt - u0);
   const int i = pi / F, j = pi % F;
-  for (int b = threadIdx.x; b < kSampleBins; b += kSampleThreads) h[b] = 0u;
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int r = 0; r < rows; ++r) {
-      rstart[r] = acc;
-      const int u = u0 + r;
-      acc += min(u + s.w, nt - 1) - max(u - s.w, 0) + 1;
-    }
-    rstart[rows] = acc;
-  }
-  __syncthreads();
-  const int shift = sample_shift(p.pass), width = sample_width(p.pass);
-  const int hi_shift = shift + width;   // digits above this one must match the prefix
-  const int total = rstart[rows];
-  int r = 0;
-  for (int f = threadIdx.x; f < total; f += kSampleThreads) {
-    while (r + 1 < rows && rstart[r + 1] <= f) ++r;   // f increases per thread
-    const int u = u0 + r;
-    const int v = max(u - s.w, 0) + (f - rstart[r]);
-    const uint64_t key = sample_key(p.seed, F, nt, i, j, u, v);
-    const bool match = hi_shift >= 64 || ((key ^ s.prefix) >> hi_shift) == 0ull;
-    if (match) atomicAdd(&h[(key >> shift) & ((1ull << width) - 1ull)], 1u);
-  }
-  __syncthreads();
-  uint32_t* gh = p.hist + static_cast<int64_t>(pi) * kSampleBins;
-  for (int b = threadIdx.x; b < kSampleBins; b += kSampleThreads)
-    if (h[b] != 0u) atomicAdd(&gh[b], h[b]);
-}
-
-// Per frame pair: the digit whose bin holds the rank-th key; clears the bins.
-__global__ void __launch_bounds__(kSampleThreads) sample_pick_kernel(SampleParams p) {
-  constexpr int kPer = kSampleBins / kSampleThreads;   // 8 bins per thread
-  __shared__ uint64_t wsum[kSampleThreads / 32];
-  __shared__ int found_bin;
-  __shared__ uint64_t found_below;
-  const int pi = blockIdx.x;
-  SamplePair s = p.pairs[pi];
-  if (!s.active) return;
-  uint32_t* gh = p.hist + static_cast<int64_t>(pi) * kSampleBins;
-  const int width = sample_width(p.pass), shift = sample_shift(p.pass);
-  const int nbins = 1 << width;
-  uint32_t c[kPer];
-  uint64_t local = 0;
-#pragma unroll
-  for (int x = 0; x < kPer; ++x) {
-    const int b = threadIdx.x * kPer + x;
-    c[x] = b < nbins ? gh[b] : 0u;
-    local += c[x];
-  }
-  // exclusive prefix of the per-thread sums (bins ascending = keys ascending)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint64_t incl = local;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const uint64_t y = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += y;
-  }
-  if (lane == 31) wsum[warp] = incl;
-  if (threadIdx.x == 0) found_bin = -1;
-  __syncthreads();
-  uint64_t base = 0;
-  for (int w = 0; w < warp; ++w) base += wsum[w];
-  const uint64_t excl = base + incl - local;
-  if (s.rank > excl && s.rank <= excl + local) {
-    uint64_t run = excl;
+  const unsigned long long nb_below = p.below[pi], nb_win = p.inwin[pi];
+  const bool pooled = s.cap > 0u && nb_win <= s.cap && s.k > nb_below && s.k - nb_below <= nb_win;
+  unsigned long long rank = pooled ? s.k - nb_below : s.k;   // 1-based, among the keys searched
+  uint64_t prefix = 0ull;
+  for (int pass = 0; pass < kSamplePasses; ++pass) {
+    const int shift = sample_shift(pass), width = sample_width(pass);
+    const int hi_shift = shift + width;   // digits above this one must match the prefix
+    const uint64_t mask = (1ull << width) - 1ull;
+    for (int b = threadIdx.x; b < kSampleBins; b += kSampleThreads) h[b] = 0u;
+    if (threadIdx.x == 0) found_bin = -1;
+    __syncthreads();
+    if (pooled) {
+      for (uint64_t x = threadIdx.x; x < nb_win; x += kSampleThreads) {
+        const uint64_t key = p.pool[s.off + x];
+        if (hi_shift >= 64 || ((key ^ prefix) >> hi_shift) == 0ull) atomicAdd(&h[(key >> shift) & mask], 1u);
+      }
+    } else {
+      for (int u = warp; u < nt; u += kSampleThreads / 32) {
+        const int v1 = min(u + s.w, nt - 1);
+        for (int v = max(u - s.w, 0) + lane; v <= v1; v += 32) {
+          const uint64_t key = sample_key(p.seed, F, nt, i, j, u, v);
+          if (hi_shift >= 64 || ((key ^ prefix) >> hi_shift) == 0ull) atomicAdd(&h[(key >> shift) & mask], 1u);
+        }
+      }
+    }
+    __syncthreads();
+    // the bin holding the rank-th key: exclusive prefix of per-thread sums
+    // (bins ascending = keys ascending)
+    uint32_t c[kPer];
+    unsigned long long local = 0;
 #pragma unroll
     for (int x = 0; x < kPer; ++x) {
-      if (s.rank <= run + c[x]) {
-        found_bin = threadIdx.x * kPer + x;
-        found_below = run;
-        break;
-      }
-      run += c[x];
+      const int b = threadIdx.x * kPer + x;
+      c[x] = b <= static_cast<int>(mask) ? h[b] : 0u;
+      local += c[x];
     }
-  }
-  __syncthreads();
+    unsigned long long incl = local;
 #pragma unroll
-  for (int x = 0; x < kPer; ++x) {
-    const int b = threadIdx.x * kPer + x;
-    if (b < nbins) gh[b] = 0u;
-  }
-  if (threadIdx.x == 0) {
-    if (found_bin < 0) {   // the histogram does not hold rank keys: cannot happen
-      record_error(DYNRAD_ERR_DEVICE);
-      s.active = 0;
-    } else {
-      s.prefix |= static_cast<uint64_t>(found_bin) << shift;
-      s.rank -= found_below;
+    for (int off = 1; off < 32; off <<= 1) {
+      const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
     }
-    p.pairs[pi] = s;
-    if (p.pass == kSamplePasses - 1 && s.active) p.thresholds[pi] = s.prefix;
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    unsigned long long base = 0;
+    for (int x = 0; x < warp; ++x) base += wsum[x];
+    const unsigned long long excl = base + incl - local;
+    if (rank > excl && rank <= excl + local) {
+      unsigned long long run = excl;
+#pragma unroll
+      for (int x = 0; x < kPer; ++x) {
+        if (rank <= run + c[x]) {
+          found_bin = threadIdx.x * kPer + x;
+          found_below = run;
+          break;
+        }
+        run += c[x];
+      }
+    }
+    __syncthreads();
+    const int bin = found_bin;
+    const unsigned long long below_bin = found_below;
+    if (bin < 0) {   // the keys searched do not hold rank keys: cannot happen
+      if (threadIdx.x == 0) record_error(DYNRAD_ERR_DEVICE);
+      return;        // T stays UINT64_MAX
+    }
+    prefix |= static_cast<uint64_t>(bin) << shift;
+    rank -= below_bin;
+    __syncthreads();   // h, wsum and found_* are rewritten by the next pass
   }
+  if (threadIdx.x == 0) p.thresholds[pi] = prefix;
 }
 
 // Per query block I: for each candidate block J (ascending), J is kept if it
@@ -239,6 +328,7 @@ __global__ void __launch_bounds__(kSampleThreads) sample_mark_kernel(SampleParam
   }
   const int flo = p.forced_lo[I], fhi = p.forced_hi[I];
   const double need_links = g.theta_c * nI;
+  const uint64_t ustep = static_cast<uint64_t>(g.nt) * kSplitMixGamma;   // u -> u + 1
   for (int c = warp; c < nc; c += kSampleThreads / 32) {
     const int J = p.cand_col[c_beg + c];
     bool kp = J >= flo && J <= fhi;
@@ -251,15 +341,25 @@ __global__ void __launch_bounds__(kSampleThreads) sample_mark_kernel(SampleParam
         uint32_t cnt = 0;
         if (k < k1) {
           const int j = k / g.nt, v = k % g.nt;
-          for (int q = q0; q < q1; ++q) {
-            const int i = q / g.nt, u = q % g.nt;
+          // I's tokens in runs of one frame i; in each run only the u within
+          // w(t) of v are in P(i, j)
+          for (int q = q0; q < q1;) {
+            const int i = q / g.nt, ua = q % g.nt;
+            const int qe = min(q1, (i + 1) * g.nt);
             const int t = i > j ? i - j : j - i;
-            const int d = u > v ? u - v : v - u;
-            if (!rt[t] || d > wt[t]) continue;   // not in P(i, j)
-            if (t >= 2 &&
-                sample_key(p.seed, g.frames, g.nt, i, j, u, v) > p.thresholds[static_cast<int64_t>(i) * g.frames + j])
-              continue;                          // not sampled
-            ++cnt;
+            if (rt[t]) {
+              const int lo = max(ua, v - wt[t]), hi = min(ua + (qe - q) - 1, v + wt[t]);
+              if (lo <= hi) {
+                if (t < 2) {
+                  cnt += hi - lo + 1;   // no sampling at t <= 1
+                } else {
+                  const uint64_t T = p.thresholds[static_cast<int64_t>(i) * g.frames + j];
+                  uint64_t z = sample_state(p.seed, g.frames, g.nt, i, j, lo, v);
+                  for (int u = lo; u <= hi; ++u, z += ustep) cnt += splitmix64_mix(z) <= T ? 1u : 0u;
+                }
+              }
+            }
+            q = qe;
           }
         }
         n_active += __popc(__ballot_sync(0xffffffffu, k < k1 && static_cast<double>(cnt) > need_links));

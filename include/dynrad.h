@@ -231,9 +231,14 @@ int dynrad_sparse_attn(const void *q, const void *k, const void *v, int32_t B,
  * seeded with `seed`, c = ((i*F + j)*N_t + u)*N_t + v (keys never tie).  The
  * sampled token links are aggregated to blocks with (theta_c, theta_m) as for
  * the candidate set (Sec. 3.1) and united with each row's forced range.  The
- * mask is a subset of the candidate set; building it costs a few radix passes
- * over all candidate token pairs (cache it: it depends only on the geometry,
- * rho1, rho2 and seed).
+ * mask is a subset of the candidate set; building it costs one pass over all
+ * candidate token pairs, which pools the keys near each frame pair's expected
+ * k-th key, then a radix select per frame pair over its pooled keys (cache the
+ * mask: it depends only on the geometry, rho1, rho2 and seed).  T(i, j) is
+ * exact whatever the pool size: a frame pair whose pool slots do not fit in
+ * the workspace, or whose k-th key falls outside its pooled range, is
+ * selected by radix passes that recompute all of its keys (one CTA per pair,
+ * much slower).
  *
  *   geom, cand_*, forced_*  the geometry and its candidate set / forced ranges
  *                 from dynrad_build_candidates (DEVICE)
@@ -247,8 +252,12 @@ int dynrad_sparse_attn(const void *q, const void *k, const void *v, int32_t B,
  *                 key of frame pair (i, j) (row-major i*F + j); UINT64_MAX
  *                 where no sampling happens (t <= 1, pairs the split rule
  *                 drops)
- *   workspace     DEVICE, 256-byte aligned, dynrad_sampled_mask_workspace_bytes
- *                 (geom, cand_nnz) bytes
+ *   workspace     DEVICE, 256-byte aligned, workspace_bytes long:
+ *                 dynrad_sampled_mask_workspace_bytes(geom, cand_nnz) bytes
+ *                 give every frame pair its pool; any size down to
+ *                 dynrad_sampled_mask_workspace_min_bytes(geom, cand_nnz) is
+ *                 accepted (the same result; frame pairs left without pool
+ *                 slots take the slow exact path)
  * Errors: DYNRAD_ERR_INVALID_ARG (null pointer, rho out of range, replicas <
  * 1, misaligned workspace), DYNRAD_ERR_UNSUPPORTED (block not 32/64/128, size
  * limits), DYNRAD_ERR_CAPACITY (workspace) -- before any launch; a col_idx
@@ -256,6 +265,8 @@ int dynrad_sparse_attn(const void *q, const void *k, const void *v, int32_t B,
  */
 size_t dynrad_sampled_mask_workspace_bytes(const dynrad_geom *geom,
                                            int64_t cand_nnz);
+size_t dynrad_sampled_mask_workspace_min_bytes(const dynrad_geom *geom,
+                                               int64_t cand_nnz);
 int dynrad_build_sampled_mask(const dynrad_geom *geom, double rho1, double rho2,
                               uint64_t seed, const int32_t *cand_row_ptr,
                               const int32_t *cand_col, int64_t cand_nnz,

@@ -2,6 +2,7 @@
 every symbol include/dynrad.h declares, and rejects bad arguments before any
 device work."""
 import ctypes
+import math
 import os
 import re
 
@@ -9,6 +10,7 @@ import pytest
 
 from block_sparse_attention_candidate_b200 import abi
 from block_sparse_attention_candidate_b200.workloads import WORKLOADS, Geometry
+from oracle import geometry
 
 HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "dynrad.h")
 
@@ -213,9 +215,25 @@ def test_sampled_mask_argument_errors_before_launch():
     g16 = abi.make_geom(Geometry(4, 4, 4, 16, 0.5, 2.0))
     assert call(geom_=g16) == abi.DYNRAD_ERR_UNSUPPORTED
     F = geom.frames
+    least = L.dynrad_sampled_mask_workspace_min_bytes(ctypes.byref(g), 100)
+    # frame-pair records (56 B), two counters each plus one, thresholds, kept lists, scan partials
+    fixed = F * F * (56 + 16 + 8) + 8 + 400 + 8
+    assert fixed <= least < fixed + 256 * 5
+    assert call(ws_bytes=least - 1) == abi.DYNRAD_ERR_CAPACITY
+    # the pool: per sampled frame pair, slots for its widest key window
+    w, r = geometry.frame_tables(geom)
+    nt = geom.tokens_per_frame
+    keys = 0
+    for t in range(2, F):
+        if not r[t]:
+            continue
+        wc = min(int(w[t]), nt - 1)
+        n = nt * (2 * wc + 1) - wc * (wc + 1)
+        e = 7.0 * math.sqrt(n) + 128.0
+        slots = min(n, math.ceil(e + 8.0 * math.sqrt(e) + 64.0), 2 ** 31 - 1)
+        keys += 2 * (F - t) * (slots + 2)
     need = L.dynrad_sampled_mask_workspace_bytes(ctypes.byref(g), 100)
-    # frame-pair records (48 B), 2048-bin histograms, thresholds, kept lists, scan partials
-    assert F * F * (48 + 2048 * 4 + 8) + 400 <= need < F * F * (48 + 2048 * 4 + 8) + 400 + 256 * 6
+    assert least + 8 * keys <= need < least + 8 * keys + 256
 
 
 def test_token_mask_argument_errors_before_launch():

@@ -107,3 +107,48 @@ def test_attention_over_the_sampled_mask_tiny():
         lcol = col_np[rp_np[h * nb]:rp_np[(h + 1) * nb]]
         o_ref[0, h], lse_ref[0, h] = OA.sparse_attention(qh, kh, vh, wl.geom.block, lrp, lcol)
     compare_attention(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, "sampled static")
+
+
+def _ws_sizes(geom, cand):
+    import ctypes
+    L = abi.lib()
+    g = abi.make_geom(geom)
+    least = int(L.dynrad_sampled_mask_workspace_min_bytes(ctypes.byref(g), cand["nnz"]))
+    full = int(L.dynrad_sampled_mask_workspace_bytes(ctypes.byref(g), cand["nnz"]))
+    assert 0 < least < full
+    return least, full
+
+
+@pytest.mark.parametrize("name", ["small0", "small3", "wan13b_480p"])
+def test_pool_size_does_not_change_the_result(name):
+    # no pool (every frame pair recomputes its keys in each radix pass), half a
+    # pool (some pooled, some not) and the full pool give the same T and mask
+    geom = SMALL[int(name[5:])] if name.startswith("small") else WORKLOADS[name].geom
+    rho1, rho2, seed = 0.3, 0.1, 77
+    cand = abi.dynrad_build_candidates(geom)
+    least, full = _ws_sizes(geom, cand)
+    outs = []
+    for ws in (least, least + (full - least) // 2, full):
+        rp, col, thr = abi.dynrad_build_sampled_mask(geom, cand, rho1, rho2, seed, thresholds=True,
+                                                     workspace_bytes=ws)
+        torch.cuda.synchronize()
+        check_device_status()
+        rp = rp.cpu().numpy().astype(np.int64)
+        outs.append((rp, col.cpu().numpy().astype(np.int64)[: rp[-1]], thr.cpu().numpy().view(np.uint64)))
+    for rp, col, thr in outs[:2]:
+        np.testing.assert_array_equal(thr, outs[2][2])
+        np.testing.assert_array_equal(rp, outs[2][0])
+        np.testing.assert_array_equal(col, outs[2][1])
+    if name.startswith("small"):
+        F = geom.frames
+        for i in range(F):
+            for j in range(F):
+                _, _, T = OSm.frame_pair_threshold(geom, i, j, rho1, rho2, seed)
+                want = np.uint64(2 ** 64 - 1) if T is None else np.uint64(T)
+                assert outs[0][2][i * F + j] == want, (i, j)
+    else:
+        F = geom.frames
+        for i, j in [(0, 2), (F - 1, 0), (5, 17)]:
+            _, _, T = OSm.frame_pair_threshold(geom, i, j, rho1, rho2, seed)
+            want = np.uint64(2 ** 64 - 1) if T is None else np.uint64(T)
+            assert outs[0][2][i * F + j] == want, (i, j)
