@@ -165,8 +165,12 @@ __global__ void sample_setup_kernel(SampleParams p) {
 // One pass over the keys of frame pair blockIdx.x, rows u in
 // [blockIdx.y * 64, +64), one warp per row (lanes over v): counts the keys
 // below the pair's window and appends the keys inside it to the pair's pool
-// slots (in any order).
+// slots (in any order).  Each warp gathers its window keys in shared memory
+// and claims pool slots for them in one atomic when its buffer fills or its
+// rows are done.
 __global__ void __launch_bounds__(kSampleThreads) sample_collect_kernel(SampleParams p) {
+  constexpr int kBuf = 64;   // window keys buffered per warp
+  __shared__ uint64_t wbuf[kSampleThreads / 32][kBuf];
   __shared__ unsigned long long wsum[kSampleThreads / 32];
   const int F = p.g.frames, nt = p.g.nt;
   const int pi = blockIdx.x;
@@ -177,7 +181,20 @@ __global__ void __launch_bounds__(kSampleThreads) sample_collect_kernel(SamplePa
   const int u1 = min(u0 + kSampleRowsPerCta, nt);
   const int i = pi / F, j = pi % F;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned lt = (1u << lane) - 1u;
   const uint64_t step = 32ull * kSplitMixGamma;
+  uint64_t* buf = wbuf[warp];
+  uint32_t nbuf = 0;   // warp-uniform
+  auto flush = [&]() {
+    __syncwarp();
+    unsigned long long base = 0;
+    if (lane == 0) base = atomicAdd(&p.inwin[pi], static_cast<unsigned long long>(nbuf));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    for (uint32_t x = lane; x < nbuf; x += 32)
+      if (base + x < s.cap) p.pool[s.off + base + x] = buf[x];   // beyond cap: the select falls back
+    __syncwarp();
+    nbuf = 0;
+  };
   uint32_t below = 0;
   for (int u = u0 + warp; u < u1; u += kSampleThreads / 32) {   // warp-uniform
     const int va = max(u - s.w, 0), vb = min(u + s.w, nt - 1);
@@ -189,17 +206,13 @@ __global__ void __launch_bounds__(kSampleThreads) sample_collect_kernel(SamplePa
       const bool in_win = valid && key >= s.lo && key <= s.hi;
       const unsigned m = __ballot_sync(0xffffffffu, in_win);
       if (m != 0u) {
-        const int leader = __ffs(m) - 1;
-        unsigned long long base = 0;
-        if (lane == leader) base = atomicAdd(&p.inwin[pi], static_cast<unsigned long long>(__popc(m)));
-        base = __shfl_sync(0xffffffffu, base, leader);
-        if (in_win) {
-          const unsigned long long pos = base + __popc(m & ((1u << lane) - 1u));
-          if (pos < s.cap) p.pool[s.off + pos] = key;   // beyond cap: the select falls back
-        }
+        if (nbuf + __popc(m) > kBuf) flush();
+        if (in_win) buf[nbuf + __popc(m & lt)] = key;
+        nbuf += __popc(m);
       }
     }
   }
+  if (nbuf != 0u) flush();
   unsigned long long bsum = below;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) bsum += __shfl_xor_sync(0xffffffffu, bsum, o);
