@@ -2,12 +2,15 @@
 // overlapped with the kernels (a runtime convenience; the paper has no
 // counterpart).
 //
-// The B*H (batch, head) rows of the layer are cut into chunks.  Three queues
+// The B*H (batch, head) rows of the layer are cut into chunks.  Four queues
 // run at once: a copy-in stream moves the chunks' Q, K, V into the device
-// workspace, the caller's stream runs stages 2 and 3 of every run on each chunk
-// as soon as its inputs are in, and a copy-out stream returns each (chunk, run)
-// O and LSE as soon as its attention kernel is done.  PCIe is full duplex, so
-// with enough chunks the copies hide behind the kernels except for the first
+// workspace; two compute queues (the caller's stream and a second one) take
+// the (chunk, run) items in turn and run stages 2 and 3 of each as soon as its
+// chunk's inputs are in, each queue with its own kept CSR and selection
+// workspace, so one item's kernels start while the previous item's attention
+// kernel drains its last wave; and a copy-out stream returns each item's O and
+// LSE as soon as its attention kernel is done.  PCIe is full duplex, so with
+// enough chunks the copies hide behind the kernels except for the first
 // chunk's copy-in and the last chunk's copy-out, which the schedule keeps small
 // (chunks of 1 and 2 rows at both ends).
 //
@@ -34,8 +37,8 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 struct HostLayout {
   size_t q = 0, k = 0, v = 0;   // full [B*H, N, D] inputs
   std::vector<size_t> o, lse;   // per run, full outputs
-  size_t row_ptr = 0, col = 0;  // one kept CSR for a chunk (largest run)
-  size_t sel = 0;               // one selection workspace for a chunk (largest run)
+  size_t row_ptr[2] = {0, 0}, col[2] = {0, 0};  // per compute queue: a chunk's kept CSR (largest run)
+  size_t sel[2] = {0, 0};                       // per compute queue: a chunk's selection workspace
   size_t sel_bytes = 0, col_cap = 0;
   size_t total = 0;
 };
@@ -73,13 +76,15 @@ bool host_layout(int32_t B, int32_t H, int32_t N, int32_t D, const dynrad_host_r
     L.lse.push_back(off);
     off += align256(static_cast<size_t>(bh) * N * 4);
   }
-  L.row_ptr = off;
-  off += align256(static_cast<size_t>(chunk * max_nb + 1) * 4);
-  L.col = off;
-  off += align256(static_cast<size_t>(max_col) * 4);
+  for (int x = 0; x < 2; ++x) {
+    L.row_ptr[x] = off;
+    off += align256(static_cast<size_t>(chunk * max_nb + 1) * 4);
+    L.col[x] = off;
+    off += align256(static_cast<size_t>(max_col) * 4);
+    L.sel[x] = off;
+    off += align256(max_sel);
+  }
   L.col_cap = static_cast<size_t>(max_col);
-  L.sel = off;
-  off += align256(max_sel);
   L.sel_bytes = max_sel;
   L.total = off;
   *out = L;
@@ -89,12 +94,12 @@ bool host_layout(int32_t B, int32_t H, int32_t N, int32_t D, const dynrad_host_r
 // Streams and events made for one call; released when the call returns (the
 // runtime defers the release of objects with work still pending).
 struct CallObjects {
-  cudaStream_t in = nullptr, out = nullptr;
+  cudaStream_t in = nullptr, out = nullptr, comp = nullptr;
   std::vector<cudaEvent_t> events;
   ~CallObjects() {
     for (cudaEvent_t e : events) cudaEventDestroy(e);
-    if (in != nullptr) cudaStreamDestroy(in);
-    if (out != nullptr) cudaStreamDestroy(out);
+    for (cudaStream_t s : {in, out, comp})
+      if (s != nullptr) cudaStreamDestroy(s);
   }
   cudaEvent_t event() {
     cudaEvent_t e = nullptr;
@@ -106,14 +111,14 @@ struct CallObjects {
 
 // Joins the side streams back into the caller's stream when the call returns,
 // on every path once they exist: whatever was queued on them (copies into the
-// workspace from the caller's host buffers, copies out to them) is then ordered
-// before anything the caller queues next, even after an error return.  If an
-// event cannot be made, it falls back to waiting on the host.
+// workspace from the caller's host buffers, kernels, copies out to them) is
+// then ordered before anything the caller queues next, even after an error
+// return.  If an event cannot be made, it falls back to waiting on the host.
 struct JoinOnReturn {
   cudaStream_t main;
   CallObjects* co;
   ~JoinOnReturn() {
-    for (cudaStream_t side : {co->in, co->out}) {
+    for (cudaStream_t side : {co->in, co->comp, co->out}) {
       if (side == nullptr) continue;
       cudaEvent_t e = co->event();
       if (e == nullptr || cudaEventRecord(e, side) != cudaSuccess || cudaStreamWaitEvent(main, e, 0) != cudaSuccess)
@@ -183,13 +188,15 @@ int dynrad_host_path(const void* q_host, const void* k_host, const void* v_host,
   // declared after co: joins the side streams before co releases them
   JoinOnReturn join{main, &co};
   if (cudaStreamCreateWithFlags(&co.in, cudaStreamNonBlocking) != cudaSuccess ||
-      cudaStreamCreateWithFlags(&co.out, cudaStreamNonBlocking) != cudaSuccess)
+      cudaStreamCreateWithFlags(&co.out, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&co.comp, cudaStreamNonBlocking) != cudaSuccess)
     return DYNRAD_ERR_CUDA;
-  // both side streams start after everything already queued on the caller's
+  // the side streams start after everything already queued on the caller's
   // stream (an earlier call may still read this workspace)
   cudaEvent_t start = co.event();
   if (start == nullptr || cudaEventRecord(start, main) != cudaSuccess ||
-      cudaStreamWaitEvent(co.in, start, 0) != cudaSuccess || cudaStreamWaitEvent(co.out, start, 0) != cudaSuccess)
+      cudaStreamWaitEvent(co.in, start, 0) != cudaSuccess || cudaStreamWaitEvent(co.out, start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(co.comp, start, 0) != cudaSuccess)
     return DYNRAD_ERR_CUDA;
 
   // copy-in of every chunk, in order
@@ -207,29 +214,35 @@ int dynrad_host_path(const void* q_host, const void* k_host, const void* v_host,
     if (in_done[c] == nullptr || cudaEventRecord(in_done[c], co.in) != cudaSuccess) return DYNRAD_ERR_CUDA;
   }
 
-  // kernels per chunk on the caller's stream; copy-out per (chunk, run)
-  int32_t* row_ptr = reinterpret_cast<int32_t*>(ws + L.row_ptr);
-  int32_t* col = reinterpret_cast<int32_t*>(ws + L.col);
+  // (chunk, run) items alternate between the two compute queues, each with
+  // its own kept CSR and selection workspace; copy-out per item
+  const cudaStream_t queue[2] = {main, co.comp};
+  int64_t item = 0;
   for (int64_t c = 0; c < n_chunks; ++c) {
     const int64_t r0 = sched[c].first, rows = sched[c].second;
-    if (cudaStreamWaitEvent(main, in_done[c], 0) != cudaSuccess) return DYNRAD_ERR_CUDA;
     const uint8_t* qc = ws + L.q + r0 * row_in;
     const uint8_t* kc = ws + L.k + r0 * row_in;
     const uint8_t* vc = ws + L.v + r0 * row_in;
-    for (int r = 0; r < n_runs; ++r) {
+    for (int r = 0; r < n_runs; ++r, ++item) {
       const dynrad_host_run& run = runs[r];
+      const int x = static_cast<int>(item & 1);
+      const cudaStream_t s = queue[x];
+      const dynrad_stream_t ss = reinterpret_cast<dynrad_stream_t>(s);
+      int32_t* row_ptr = reinterpret_cast<int32_t*>(ws + L.row_ptr[x]);
+      int32_t* col = reinterpret_cast<int32_t*>(ws + L.col[x]);
+      if (cudaStreamWaitEvent(s, in_done[c], 0) != cudaSuccess) return DYNRAD_ERR_CUDA;
       int rc = dynrad_select_blocks(qc, kc, 1, static_cast<int32_t>(rows), N, D, &run.geom, run.cand_row_ptr,
                                     run.cand_col, run.cand_nnz, run.cand_max_row, run.forced_lo, run.forced_hi,
                                     run.mode, run.rho_or_tau, row_ptr, col, static_cast<int64_t>(L.col_cap),
-                                    nullptr, ws + L.sel, L.sel_bytes, stream);
+                                    nullptr, ws + L.sel[x], L.sel_bytes, ss);
       if (rc != DYNRAD_OK) return rc;
       uint8_t* oc = ws + L.o[r] + r0 * row_in;
       float* lc = reinterpret_cast<float*>(ws + L.lse[r] + r0 * row_lse);
       rc = dynrad_sparse_attn(qc, kc, vc, 1, static_cast<int32_t>(rows), N, D, run.geom.block, row_ptr, col,
-                              scale, oc, lc, stream);
+                              scale, oc, lc, ss);
       if (rc != DYNRAD_OK) return rc;
       cudaEvent_t done = co.event();
-      if (done == nullptr || cudaEventRecord(done, main) != cudaSuccess ||
+      if (done == nullptr || cudaEventRecord(done, s) != cudaSuccess ||
           cudaStreamWaitEvent(co.out, done, 0) != cudaSuccess)
         return DYNRAD_ERR_CUDA;
       if (cudaMemcpyAsync(static_cast<uint8_t*>(run.o_host) + r0 * row_in, oc, rows * row_in,

@@ -28,8 +28,8 @@
  *     attended, padded query rows are never written).  Nb = ceil(N / block).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) unless stated.  The library allocates no memory and frees none of
- *     the caller's (dynrad_host_path creates, and releases, two streams and a
- *     few events per call).
+ *     the caller's (dynrad_host_path creates, and releases, three streams and
+ *     a few events per call).
  *   - Every call returns a dynrad_status.  Argument errors are found on the
  *     host before any launch.  Errors found by a kernel (capacity exceeded, a
  *     bounded wait that ran out) are recorded in a device status word read by
@@ -334,8 +334,10 @@ int dynrad_build_token_mask(const void *q, const void *k, int32_t B, int32_t H,
  * (as dynrad_select_blocks) and the attention output (as dynrad_sparse_attn)
  * and writes the run's O and LSE to host memory.  The B*H (batch, head) rows
  * go through in chunks of chunk_bh rows: the copy-in of later chunks, the
- * kernels of the current chunk and the copy-out of finished (chunk, run)
- * outputs run concurrently on two streams the call creates and on `stream`.
+ * kernels of the current (chunk, run) items and the copy-out of finished
+ * items run concurrently on three streams the call creates and on `stream`
+ * (items alternate between `stream` and one created compute stream, so one
+ * item's kernels start while the previous item's attention drains).
  * Results are bit-identical to the device-resident calls (every stage is
  * independent per (batch, head) row).
  *
@@ -357,8 +359,8 @@ int dynrad_build_token_mask(const void *q, const void *k, int32_t B, int32_t H,
  *   scale         as for dynrad_sparse_attn (0 means 1/sqrt(D))
  *   workspace     DEVICE, 256-byte aligned, at least
  *                 dynrad_host_path_workspace_bytes(...) bytes: it holds Q, K, V,
- *                 every run's O and LSE, and one chunk's kept CSR and
- *                 selection workspace
+ *                 every run's O and LSE, and per compute stream one chunk's
+ *                 kept CSR and selection workspace
  *
  * Ordering: the call's device work starts after the work already queued on
  * `stream` and `stream` continues only after the last copy-out, so back-to-

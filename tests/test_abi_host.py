@@ -189,8 +189,9 @@ def test_host_path_workspace_size_formula():
     got = L.dynrad_host_path_workspace_bytes(B, H, N, D, runs, 4, chunk)
     qkv = B * H * N * D * 2
     sel = abi.dynrad_select_workspace_bytes(1, chunk, N, D, g, nnz)
-    # Q, K, V; O and LSE per run; one chunk's kept CSR and selection workspace
-    need = 3 * qkv + 4 * (qkv + B * H * N * 4) + (chunk * g.n_blocks + 1) * 4 + chunk * nnz * 4 + sel
+    # Q, K, V; O and LSE per run; per compute stream one chunk's kept CSR and
+    # selection workspace
+    need = 3 * qkv + 4 * (qkv + B * H * N * 4) + 2 * ((chunk * g.n_blocks + 1) * 4 + chunk * nnz * 4 + sel)
     assert need <= got < need + 256 * 16
 
 
