@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <vector>
@@ -519,7 +520,7 @@ int dynrad_select_blocks(const void* q, const void* k, int32_t B, int32_t H, int
 namespace {
 
 struct SampleWorkspace {
-  size_t pairs, counters, thresholds, kept, partial, pool, total;
+  size_t pairs, counters, thresholds, kept, keep, partial, pool, total;
 };
 
 // Pool slots for every sampled frame pair at its largest window (q = 1/2):
@@ -544,9 +545,10 @@ SampleWorkspace sample_layout(const GeomDev& g, int64_t cand_nnz, bool with_pool
   const int64_t tiles = (g.nb + 1 + kScanTile - 1) / kScanTile;
   w.pairs = 0;
   w.counters = align256(w.pairs + static_cast<size_t>(fp) * sizeof(SamplePair));
-  w.thresholds = align256(w.counters + static_cast<size_t>(2 * fp + 1) * 8);
+  w.thresholds = align256(w.counters + static_cast<size_t>(2 * fp + 2) * 8);
   w.kept = align256(w.thresholds + static_cast<size_t>(fp) * 8);
-  w.partial = align256(w.kept + static_cast<size_t>(cand_nnz) * 4);
+  w.keep = align256(w.kept + static_cast<size_t>(cand_nnz) * 4);
+  w.partial = align256(w.keep + static_cast<size_t>(cand_nnz));
   w.pool = align256(w.partial + static_cast<size_t>(tiles) * 8);
   w.total = with_pool ? align256(w.pool + static_cast<size_t>(sample_pool_keys(g)) * 8) : w.pool;
   return w;
@@ -583,8 +585,8 @@ int dynrad_build_sampled_mask(const dynrad_geom* geom, double rho1, double rho2,
   if (g.block != 32 && g.block != 64 && g.block != 128) return DYNRAD_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(replicas) * g.nb + 1 > INT32_MAX) return DYNRAD_ERR_UNSUPPORTED;
   if ((static_cast<int64_t>(g.nt) + kSampleRowsPerCta - 1) / kSampleRowsPerCta > 65535) return DYNRAD_ERR_UNSUPPORTED;
-  // the marking keeps a frame table and one flag per candidate in default shared memory
-  if (static_cast<size_t>(g.frames) * 5 + static_cast<size_t>(g.nb) + 16 > 48 * 1024) return DYNRAD_ERR_UNSUPPORTED;
+  // the marking keeps a frame table in default shared memory
+  if (static_cast<size_t>(g.frames) * 5 + 16 > 48 * 1024) return DYNRAD_ERR_UNSUPPORTED;
   const SampleWorkspace w = sample_layout(g, cand_nnz, false);
   if (workspace_bytes < w.total) return DYNRAD_ERR_CAPACITY;
   cudaStream_t st = as_stream(stream);
@@ -599,6 +601,9 @@ int dynrad_build_sampled_mask(const dynrad_geom* geom, double rho1, double rho2,
   sp.below = reinterpret_cast<unsigned long long*>(ws + w.counters);
   sp.inwin = sp.below + fp;
   sp.pool_used = sp.inwin + fp;
+  sp.mark_ticket = sp.pool_used + 1;
+  sp.cand_nnz = cand_nnz;
+  sp.keep = ws + w.keep;
   sp.pool = reinterpret_cast<uint64_t*>(ws + w.pool);
   sp.pool_cap = (workspace_bytes - w.pool) / 8;   // whatever the caller gave beyond the fixed part
   sp.thresholds = reinterpret_cast<uint64_t*>(ws + w.thresholds);
@@ -608,7 +613,7 @@ int dynrad_build_sampled_mask(const dynrad_geom* geom, double rho1, double rho2,
   sp.forced_hi = forced_hi;
   sp.counts = row_ptr;
   sp.kept_tmp = reinterpret_cast<int32_t*>(ws + w.kept);
-  if (cudaMemsetAsync(sp.below, 0, static_cast<size_t>(2 * fp + 1) * 8, st) != cudaSuccess) return DYNRAD_ERR_CUDA;
+  if (cudaMemsetAsync(sp.below, 0, static_cast<size_t>(2 * fp + 2) * 8, st) != cudaSuccess) return DYNRAD_ERR_CUDA;
   sample_setup_kernel<<<(fp + 255) / 256, 256, 0, st>>>(sp);
   if ((rc = launch_status()) != DYNRAD_OK) return rc;
   const dim3 cgrid(fp, (g.nt + kSampleRowsPerCta - 1) / kSampleRowsPerCta);
@@ -616,11 +621,21 @@ int dynrad_build_sampled_mask(const dynrad_geom* geom, double rho1, double rho2,
   if ((rc = launch_status()) != DYNRAD_OK) return rc;
   sample_select_kernel<<<fp, kSampleThreads, 0, st>>>(sp);
   if ((rc = launch_status()) != DYNRAD_OK) return rc;
-  const size_t msmem = static_cast<size_t>(g.frames) * 5 + static_cast<size_t>(g.nb) + 16;
-  if (g.block == 32) sample_mark_kernel<32><<<g.nb, kSampleThreads, msmem, st>>>(sp);
-  else if (g.block == 64) sample_mark_kernel<64><<<g.nb, kSampleThreads, msmem, st>>>(sp);
-  else sample_mark_kernel<128><<<g.nb, kSampleThreads, msmem, st>>>(sp);
-  if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  // marking: warps claim candidates from a ticket; enough CTAs to fill the SMs
+  const size_t msmem = static_cast<size_t>(g.frames) * 5 + 16;
+  {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (cand_nnz + kMarkChunk * (kSampleThreads / 32) - 1) / (kMarkChunk * (kSampleThreads / 32));
+    const unsigned mgrid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(want, 6LL * sms)));
+    if (g.block == 32) sample_mark_kernel<32><<<mgrid, kSampleThreads, msmem, st>>>(sp);
+    else if (g.block == 64) sample_mark_kernel<64><<<mgrid, kSampleThreads, msmem, st>>>(sp);
+    else sample_mark_kernel<128><<<mgrid, kSampleThreads, msmem, st>>>(sp);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+    const unsigned cgrid2 = static_cast<unsigned>((static_cast<int64_t>(g.nb) * 32 + kSampleThreads - 1) / kSampleThreads);
+    sample_compact_kernel<<<cgrid2, kSampleThreads, 0, st>>>(sp);
+    if ((rc = launch_status()) != DYNRAD_OK) return rc;
+  }
   // counts -> offsets -> compacted replica 0 -> replicas
   {
     const int64_t rows = g.nb;

@@ -17,7 +17,8 @@
 // (k - 1/2) / |P| * 2^64, within a few sqrt(q (1 - q) / |P|) * 2^64 (q = k / |P|,
 // the spread of a uniform order statistic).  One pass counts the keys below a
 // window [lo, hi] around that point (7 such deviations plus 64 keys' worth on
-// each side) and copies the keys inside it to a per-pair pool; if the counts
+// each side, widened to whole multiples of 2^32 so that a key's high word
+// classifies it) and copies the keys inside it to a per-pair pool; if the counts
 // show that the window holds the k-th key, a radix select over the few
 // thousand pooled keys gives T.  Otherwise (never seen with real keys, but
 // possible for a pair whose pool reservation did not fit the workspace) the
@@ -31,8 +32,11 @@
 //                          pools the keys inside it.
 //   sample_select_kernel   per frame pair: 11-bit radix select of the k-th key
 //                          over the pooled keys (or over all keys).
-//   sample_mark_kernel     per query block, one warp per candidate block: its
-//                          token-level sampled links, (theta_c, theta_m).
+//   sample_mark_kernel     one warp per candidate block (warps claim candidates
+//                          in small chunks from a ticket): its token-level
+//                          sampled links, (theta_c, theta_m), a keep flag.
+//   sample_compact_kernel  one warp per query block: the kept candidates in
+//                          list order and the row's count.
 //   replicate_csr_kernel   copies the head-shared CSR for every (batch, head).
 #pragma once
 
@@ -89,14 +93,23 @@ struct SampleParams {
   const int32_t* cand_col;
   const int32_t* forced_lo;
   const int32_t* forced_hi;
+  int64_t cand_nnz;
+  uint8_t* keep;            // [cand_nnz] per candidate: kept (1) or not (0)
+  unsigned long long* mark_ticket;   // candidates handed out to marking warps (zeroed before setup)
   int32_t* counts;          // [nb] kept per row
   int32_t* kept_tmp;        // [cand_nnz] kept lists at the candidate offsets
 };
 
-__device__ __forceinline__ uint64_t splitmix64_mix(uint64_t z) {
+// The SplitMix64 finaliser up to its last xor-shift; splitmix64_mix is
+// y ^ (y >> 31) of this y, whose high 32 bits are yh ^ (yh >> 31), yh = y >> 32.
+__device__ __forceinline__ uint64_t splitmix64_premix(uint64_t z) {
   z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
-  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
-  return z ^ (z >> 31);
+  return (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+}
+
+__device__ __forceinline__ uint64_t splitmix64_mix(uint64_t z) {
+  const uint64_t y = splitmix64_premix(z);
+  return y ^ (y >> 31);
 }
 
 // The generator state before mixing for counter c: seed + (c + 1) * gamma
@@ -150,6 +163,10 @@ __global__ void sample_setup_kernel(SampleParams p) {
     const double two64 = 18446744073709551616.0;
     if (lo_f > 0.0) s.lo = static_cast<uint64_t>(lo_f * two64);   // lo_f < mid < 1
     if (hi_f < 1.0 - 0x1p-40) s.hi = static_cast<uint64_t>(hi_f * two64);
+    // widened to whole 2^32 ranges (at most 2 |P| / 2^32 more keys): the
+    // collect pass then classifies a key by its high 32 bits alone
+    s.lo &= ~0xFFFFFFFFull;
+    s.hi |= 0xFFFFFFFFull;
     const double span = fmin(hi_f, 1.0) - fmax(lo_f, 0.0);
     const uint64_t cap = sample_pool_slots(n, span * n);
     const unsigned long long off = atomicAdd(p.pool_used, static_cast<unsigned long long>(cap));
@@ -195,22 +212,29 @@ __global__ void __launch_bounds__(kSampleThreads) sample_collect_kernel(SamplePa
     __syncwarp();
     nbuf = 0;
   };
+  // the window is [lo_hi * 2^32, hi_hi * 2^32 + 2^32 - 1]: a key's high word
+  // decides below / inside / above
+  const uint32_t lo_hi = static_cast<uint32_t>(s.lo >> 32), hi_hi = static_cast<uint32_t>(s.hi >> 32);
   uint32_t below = 0;
+  auto visit = [&](uint64_t z, bool valid) {   // called with the whole warp
+    const uint64_t y = splitmix64_premix(z);
+    const uint32_t yh = static_cast<uint32_t>(y >> 32);
+    const uint32_t kh = yh ^ (yh >> 31);   // high word of the key
+    below += (valid && kh < lo_hi) ? 1u : 0u;
+    const bool in_win = valid && kh >= lo_hi && kh <= hi_hi;
+    const unsigned m = __ballot_sync(0xffffffffu, in_win);
+    if (m != 0u) {
+      if (nbuf + __popc(m) > kBuf) flush();
+      if (in_win) buf[nbuf + __popc(m & lt)] = y ^ (y >> 31);
+      nbuf += __popc(m);
+    }
+  };
   for (int u = u0 + warp; u < u1; u += kSampleThreads / 32) {   // warp-uniform
     const int va = max(u - s.w, 0), vb = min(u + s.w, nt - 1);
+    const int len = vb - va + 1, full = len >> 5, tail = len & 31;
     uint64_t z = sample_state(p.seed, F, nt, i, j, u, va + lane);
-    for (int v0 = va; v0 <= vb; v0 += 32, z += step) {          // warp-uniform
-      const bool valid = v0 + lane <= vb;
-      const uint64_t key = splitmix64_mix(z);
-      below += (valid && key < s.lo) ? 1u : 0u;
-      const bool in_win = valid && key >= s.lo && key <= s.hi;
-      const unsigned m = __ballot_sync(0xffffffffu, in_win);
-      if (m != 0u) {
-        if (nbuf + __popc(m) > kBuf) flush();
-        if (in_win) buf[nbuf + __popc(m & lt)] = key;
-        nbuf += __popc(m);
-      }
-    }
+    for (int it = 0; it < full; ++it, z += step) visit(z, true);   // warp-uniform
+    if (tail != 0) visit(z, lane < tail);
   }
   if (nbuf != 0u) flush();
   unsigned long long bsum = below;
@@ -313,86 +337,113 @@ __global__ void __launch_bounds__(kSampleThreads) sample_select_kernel(SamplePar
   if (threadIdx.x == 0) p.thresholds[pi] = prefix;
 }
 
-// Per query block I: for each candidate block J (ascending), J is kept if it
-// is in F_I or if, over the sampled token links of (I, J), more than
-// theta_m * n_J of J's columns are active (a column is active when more than
-// theta_c * n_I of I's tokens link to it).  One warp per candidate (eight at a
-// time): lanes take J's columns and walk I's tokens; then warp 0 writes the
-// kept candidates in list order.
+// Candidate block J of query block I is kept if it is in F_I or if, over the
+// sampled token links of (I, J), more than theta_m * n_J of J's columns are
+// active (a column is active when more than theta_c * n_I of I's tokens link
+// to it).  One warp per candidate, lanes over J's columns, each walking I's
+// tokens; warps claim chunks of kMarkChunk consecutive candidates (flattened
+// over all rows) from a ticket, so the uneven cost of candidates (t <= 1 pairs
+// are counted in closed form, far pairs token by token) evens out.
+constexpr int kMarkChunk = 4;
+
+// Row of flattened candidate c: the I with row_ptr[I] <= c < row_ptr[I + 1].
+__device__ __forceinline__ int cand_row_of(const int32_t* row_ptr, int nb, int64_t c) {
+  int lo = 0, hi = nb - 1;   // row_ptr[0] = 0 <= c
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (static_cast<int64_t>(row_ptr[mid]) <= c) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
 template <int BS>
 __global__ void __launch_bounds__(kSampleThreads) sample_mark_kernel(SampleParams p) {
   extern __shared__ __align__(16) uint8_t sm_raw[];
   const GeomDev& g = p.g;
   int* wt = reinterpret_cast<int*>(sm_raw);                    // [F]
   uint8_t* rt = reinterpret_cast<uint8_t*>(wt + g.frames);     // [F]
-  uint8_t* keep = rt + g.frames;                               // [nb] per list position
   constexpr int kColsPerLane = (BS + 31) / 32;
-  const int I = blockIdx.x;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
   build_frame_tables(g, wt, rt);
   __syncthreads();
-  const int q0 = I * BS, q1 = min(q0 + BS, g.n);
-  const int nI = q1 - q0;
-  const int c_beg = p.cand_row_ptr[I];
-  int nc = p.cand_row_ptr[I + 1] - c_beg;
-  if (nc > g.nb || nc < 0) {   // not a valid candidate row
-    if (threadIdx.x == 0) record_error(DYNRAD_ERR_CAPACITY);
-    nc = nc < 0 ? 0 : g.nb;
-  }
-  const int flo = p.forced_lo[I], fhi = p.forced_hi[I];
-  const double need_links = g.theta_c * nI;
   const uint64_t ustep = static_cast<uint64_t>(g.nt) * kSplitMixGamma;   // u -> u + 1
-  for (int c = warp; c < nc; c += kSampleThreads / 32) {
-    const int J = p.cand_col[c_beg + c];
-    bool kp = J >= flo && J <= fhi;
-    if (!kp) {
-      const int k0 = J * BS, k1 = min(k0 + BS, g.n), nJ = k1 - k0;
-      int n_active = 0;
+  const int64_t nnz = p.cand_nnz;
+  for (;;) {
+    unsigned long long c0 = 0;
+    if (lane == 0) c0 = atomicAdd(p.mark_ticket, static_cast<unsigned long long>(kMarkChunk));
+    c0 = __shfl_sync(0xffffffffu, c0, 0);
+    if (c0 >= static_cast<unsigned long long>(nnz)) break;   // warp-uniform
+    const int64_t c1 = min(static_cast<int64_t>(c0) + kMarkChunk, nnz);
+    int I = cand_row_of(p.cand_row_ptr, g.nb, static_cast<int64_t>(c0));
+    for (int64_t c = static_cast<int64_t>(c0); c < c1; ++c) {   // warp-uniform
+      while (I + 1 < g.nb && static_cast<int64_t>(p.cand_row_ptr[I + 1]) <= c) ++I;
+      const int J = p.cand_col[c];
+      bool kp = J >= p.forced_lo[I] && J <= p.forced_hi[I];
+      if (!kp && J >= 0 && J < g.nb) {
+        const int q0 = I * BS, q1 = min(q0 + BS, g.n);
+        const double need_links = g.theta_c * (q1 - q0);
+        const int k0 = J * BS, k1 = min(k0 + BS, g.n), nJ = k1 - k0;
+        int n_active = 0;
 #pragma unroll
-      for (int x = 0; x < kColsPerLane; ++x) {
-        const int k = k0 + lane + 32 * x;
-        uint32_t cnt = 0;
-        if (k < k1) {
-          const int j = k / g.nt, v = k % g.nt;
-          // I's tokens in runs of one frame i; in each run only the u within
-          // w(t) of v are in P(i, j)
-          for (int q = q0; q < q1;) {
-            const int i = q / g.nt, ua = q % g.nt;
-            const int qe = min(q1, (i + 1) * g.nt);
-            const int t = i > j ? i - j : j - i;
-            if (rt[t]) {
-              const int lo = max(ua, v - wt[t]), hi = min(ua + (qe - q) - 1, v + wt[t]);
-              if (lo <= hi) {
-                if (t < 2) {
-                  cnt += hi - lo + 1;   // no sampling at t <= 1
-                } else {
-                  const uint64_t T = p.thresholds[static_cast<int64_t>(i) * g.frames + j];
-                  uint64_t z = sample_state(p.seed, g.frames, g.nt, i, j, lo, v);
-                  for (int u = lo; u <= hi; ++u, z += ustep) cnt += splitmix64_mix(z) <= T ? 1u : 0u;
+        for (int x = 0; x < kColsPerLane; ++x) {
+          const int k = k0 + lane + 32 * x;
+          uint32_t cnt = 0;
+          if (k < k1) {
+            const int j = k / g.nt, v = k % g.nt;
+            // I's tokens in runs of one frame i; in each run only the u within
+            // w(t) of v are in P(i, j)
+            for (int q = q0; q < q1;) {
+              const int i = q / g.nt, ua = q % g.nt;
+              const int qe = min(q1, (i + 1) * g.nt);
+              const int t = i > j ? i - j : j - i;
+              if (rt[t]) {
+                const int lo = max(ua, v - wt[t]), hi = min(ua + (qe - q) - 1, v + wt[t]);
+                if (lo <= hi) {
+                  if (t < 2) {
+                    cnt += hi - lo + 1;   // no sampling at t <= 1
+                  } else {
+                    const uint64_t T = p.thresholds[static_cast<int64_t>(i) * g.frames + j];
+                    uint64_t z = sample_state(p.seed, g.frames, g.nt, i, j, lo, v);
+                    for (int u = lo; u <= hi; ++u, z += ustep) cnt += splitmix64_mix(z) <= T ? 1u : 0u;
+                  }
                 }
               }
+              q = qe;
             }
-            q = qe;
           }
+          n_active += __popc(__ballot_sync(0xffffffffu, k < k1 && static_cast<double>(cnt) > need_links));
         }
-        n_active += __popc(__ballot_sync(0xffffffffu, k < k1 && static_cast<double>(cnt) > need_links));
+        kp = static_cast<double>(n_active) > g.theta_m * nJ;
+      } else if (!kp) {
+        if (lane == 0) record_error(DYNRAD_ERR_DEVICE);   // not a block index: dropped
       }
-      kp = static_cast<double>(n_active) > g.theta_m * nJ;
+      if (lane == 0) p.keep[c] = kp ? 1 : 0;
     }
-    if (lane == 0) keep[c] = kp ? 1 : 0;
   }
-  __syncthreads();
-  if (warp == 0) {
-    int n_kept = 0;
-    for (int c0 = 0; c0 < nc; c0 += 32) {
-      const int c = c0 + lane;
-      const bool k_ = c < nc && keep[c] != 0;
-      const unsigned bal = __ballot_sync(0xffffffffu, k_);
-      if (k_) p.kept_tmp[c_beg + n_kept + __popc(bal & ((1u << lane) - 1u))] = p.cand_col[c_beg + c];
-      n_kept += __popc(bal);
-    }
-    if (lane == 0) p.counts[I] = n_kept;
+}
+
+// One warp per query block I: its kept candidates in list order at the
+// row's candidate offsets, and its count.
+__global__ void __launch_bounds__(kSampleThreads) sample_compact_kernel(SampleParams p) {
+  const int lane = threadIdx.x & 31;
+  const int I = (blockIdx.x * kSampleThreads + threadIdx.x) >> 5;
+  if (I >= p.g.nb) return;   // whole warps
+  const int c_beg = p.cand_row_ptr[I];
+  int nc = p.cand_row_ptr[I + 1] - c_beg;
+  if (c_beg < 0 || nc < 0 || static_cast<int64_t>(c_beg) + nc > p.cand_nnz) {   // not a candidate row
+    if (lane == 0) record_error(DYNRAD_ERR_CAPACITY);
+    nc = 0;
   }
+  int n_kept = 0;
+  for (int c0 = 0; c0 < nc; c0 += 32) {   // warp-uniform
+    const int c = c0 + lane;
+    const bool k_ = c < nc && p.keep[c_beg + c] != 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, k_);
+    if (k_) p.kept_tmp[c_beg + n_kept + __popc(bal & ((1u << lane) - 1u))] = p.cand_col[c_beg + c];
+    n_kept += __popc(bal);
+  }
+  if (lane == 0) p.counts[I] = n_kept;
 }
 
 // Copies replica 0 of the CSR (rows [0, nb), entries [0, nnz)) to replicas

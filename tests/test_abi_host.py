@@ -217,9 +217,10 @@ def test_sampled_mask_argument_errors_before_launch():
     assert call(geom_=g16) == abi.DYNRAD_ERR_UNSUPPORTED
     F = geom.frames
     least = L.dynrad_sampled_mask_workspace_min_bytes(ctypes.byref(g), 100)
-    # frame-pair records (56 B), two counters each plus one, thresholds, kept lists, scan partials
-    fixed = F * F * (56 + 16 + 8) + 8 + 400 + 8
-    assert fixed <= least < fixed + 256 * 5
+    # frame-pair records (56 B), two counters each plus two, thresholds, kept
+    # lists, keep flags, scan partials
+    fixed = F * F * (56 + 16 + 8) + 16 + 400 + 100 + 8
+    assert fixed <= least < fixed + 256 * 6
     assert call(ws_bytes=least - 1) == abi.DYNRAD_ERR_CAPACITY
     # the pool: per sampled frame pair, slots for its widest key window
     w, r = geometry.frame_tables(geom)
