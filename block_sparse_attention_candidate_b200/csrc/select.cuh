@@ -423,8 +423,8 @@ __device__ __forceinline__ uint32_t select_row(const Stage2Params& p, int I, int
   const int ne = (n + 31) >> 5;   // <= E
   const int flo = p.forced_lo[I], fhi = p.forced_hi[I];
   uint32_t forced = 0u, valid = 0u;
-#pragma unroll
-  for (int i = 0; i < E; ++i) if (i < ne) {
+#pragma unroll 2
+  for (int i = 0; i < ne; ++i) {
     const int c = lane + 32 * i;
     if (c < n) {
       const int J = p.cand_col[c_beg + c];
@@ -445,14 +445,14 @@ __device__ __forceinline__ uint32_t select_row(const Stage2Params& p, int I, int
   bool keep_all = false;
   if constexpr (DYN) {
     float smax = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < E; ++i) if (i < ne)
+#pragma unroll 2
+    for (int i = 0; i < ne; ++i)
       if ((valid >> i) & 1u) smax = fmaxf(smax, srow[lane + 32 * i]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, off));
     uint64_t base = 0, ztot = 0;
-#pragma unroll
-    for (int i = 0; i < E; ++i) if (i < ne) {
+#pragma unroll 2
+    for (int i = 0; i < ne; ++i) {
       if ((valid >> i) & 1u) {
         const int c = lane + 32 * i;
         const double e = exp(static_cast<double>(srow[c]) - static_cast<double>(smax));
@@ -485,8 +485,8 @@ __device__ __forceinline__ uint32_t select_row(const Stage2Params& p, int I, int
     uint32_t prefix = 0u, pmask = 0u;
     while (true) {
       uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-#pragma unroll
-      for (int i = 0; i < E; ++i) if (i < ne) {
+#pragma unroll 2
+      for (int i = 0; i < ne; ++i) {
         if ((freev >> i) & 1u) {
           const uint32_t k = order_key(srow[lane + 32 * i]);
           if ((k & pmask) == prefix) {
@@ -515,8 +515,8 @@ __device__ __forceinline__ uint32_t select_row(const Stage2Params& p, int I, int
       __syncwarp();
       // weights < 2^36 are split into 18-bit halves; each half's bin sum stays
       // below 2^32 for rows of up to 2^14 candidates
-#pragma unroll
-      for (int i = 0; i < E; ++i) if (i < ne) {
+#pragma unroll 2
+      for (int i = 0; i < ne; ++i) {
         if ((freev >> i) & 1u) {
           const int c = lane + 32 * i;
           const uint32_t k = order_key(srow[c]);
@@ -572,8 +572,8 @@ __device__ __forceinline__ uint32_t select_row(const Stage2Params& p, int I, int
   if (!cut_none) {
     uint64_t tie_run = 0;
     const uint32_t lt_mask = (1u << lane) - 1u;
-#pragma unroll
-    for (int i = 0; i < E; ++i) if (i < ne) {
+#pragma unroll 2
+    for (int i = 0; i < ne; ++i) {
       const int c = lane + 32 * i;
       const bool fr = (freev >> i) & 1u;
       const uint32_t k = fr ? order_key(srow[c]) : 0u;
@@ -622,6 +622,29 @@ __device__ __forceinline__ void select_item(const Stage2Params& p, int bh, int g
     qsT[d * kSelRows + r] = (I0 + r < nb) ? p.qbar[(static_cast<int64_t>(bh) * nb + I0 + r) * D + d] : 0.f;
   }
   __syncthreads();
+  if constexpr (!DYN) {
+    // static mode: the group's first CSR offset (heads before this one, then
+    // groups before this one) comes from the plan's per-group counts, known
+    // now; warp 0 sums them here so the loads overlap the scoring
+    if (warp == 0) {
+      int64_t before = 0, total = 0;
+      for (int x = lane; x < p.nq; x += 32) {
+        const int64_t c = p.plan_rows[x];
+        total += c;
+        if (x < grp) before += c;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        before += __shfl_xor_sync(0xffffffffu, before, o);
+        total += __shfl_xor_sync(0xffffffffu, total, o);
+      }
+      if (lane == 0) {
+        s_excl = static_cast<int64_t>(bh) * total + before;
+        if (bh == p.rows_bh - 1 && grp == p.nq - 1)
+          p.row_ptr[static_cast<int64_t>(p.rows_bh) * nb] = static_cast<int32_t>(static_cast<int64_t>(p.rows_bh) * total);
+      }
+    }
+  }
   const int c0 = p.cand_row_ptr[I0];
   {
     // Scoring: a pair of threads per two union members.  Each thread of the
@@ -724,9 +747,9 @@ __device__ __forceinline__ void select_item(const Stage2Params& p, int bh, int g
     } else if (n > 0) {
       kept = select_row<DYN, E>(p, I, n, c_beg, sc + loc, wg + loc, bins_all + warp * 512, lane);
       const int ne = (n + 31) >> 5;
-#pragma unroll
-      for (int i = 0; i < E; ++i)
-        if (i < ne) cnt += __popc(__ballot_sync(0xffffffffu, (kept >> i) & 1u));
+#pragma unroll 2
+      for (int i = 0; i < ne; ++i)
+        cnt += __popc(__ballot_sync(0xffffffffu, (kept >> i) & 1u));
     }
   }
   if (lane == 0) s_cnt[warp] = cnt;
@@ -740,9 +763,9 @@ __device__ __forceinline__ void select_item(const Stage2Params& p, int bh, int g
       int32_t* dst = p.kept_tmp + static_cast<int64_t>(bh) * p.cand_nnz + c_beg;
       const int ne = (n + 31) >> 5;
       int run = 0;
-#pragma unroll
-      for (int i = 0; i < E; ++i) {
-        if (i < ne) {
+#pragma unroll 2
+      for (int i = 0; i < ne; ++i) {
+        {
           const bool k_ = (kept >> i) & 1u;
           const unsigned bal = __ballot_sync(0xffffffffu, k_);
           if (k_) dst[run + __popc(bal & ((1u << lane) - 1u))] = p.cand_col[c_beg + lane + 32 * i];
@@ -759,34 +782,15 @@ __device__ __forceinline__ void select_item(const Stage2Params& p, int bh, int g
       for (int r = 0; r < kSelRows; ++r) tot += s_cnt[r];
       if (tot != p.plan_rows[grp]) record_error(DYNRAD_ERR_DEVICE);   // cannot happen: same rule
     }
-    if (warp == 0) {
-      int64_t before = 0, total = 0;
-      for (int x = lane; x < p.nq; x += 32) {
-        const int64_t c = p.plan_rows[x];
-        total += c;
-        if (x < grp) before += c;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        before += __shfl_xor_sync(0xffffffffu, before, o);
-        total += __shfl_xor_sync(0xffffffffu, total, o);
-      }
-      if (lane == 0) {
-        s_excl = static_cast<int64_t>(bh) * total + before;
-        if (bh == p.rows_bh - 1 && grp == p.nq - 1)
-          p.row_ptr[static_cast<int64_t>(p.rows_bh) * nb] = static_cast<int32_t>(static_cast<int64_t>(p.rows_bh) * total);
-      }
-    }
-    __syncthreads();
     if (I < nb) {
       int64_t o = s_excl;
       for (int r = 0; r < warp; ++r) o += s_cnt[r];
       if (lane == 0) p.row_ptr[static_cast<int64_t>(bh) * nb + I] = static_cast<int32_t>(o);
       const int ne = (n + 31) >> 5;
       int run = 0;
-#pragma unroll
-      for (int i = 0; i < E; ++i) {
-        if (i < ne) {
+#pragma unroll 2
+      for (int i = 0; i < ne; ++i) {
+        {
           const bool k_ = (kept >> i) & 1u;
           const unsigned bal = __ballot_sync(0xffffffffu, k_);
           if (k_) {
