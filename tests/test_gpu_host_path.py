@@ -60,6 +60,23 @@ def test_host_path_matches_device_calls(chunk):
             assert torch.equal(r["lse_host"], lse)
 
 
+def test_host_path_three_runs_alternate_queues():
+    # (chunk, run) items alternate between two compute queues, each with its own
+    # CSR and selection buffers: with three runs a queue serves different runs
+    # (different geometries and kept counts) from one chunk to the next
+    wl = WORKLOADS["wan13b_480p"]
+    host = _host_inputs(wl)
+    B, H, N, D = host["q"].shape
+    runs = _runs(wl, [("static", 0.2, None), ("dynamic", 0.8, 0.7), ("static", 0.35, 0.3)], B, H, N, D)
+    ref = _device_reference(host, runs)
+    abi.dynrad_host_path(host["q"], host["k"], host["v"], runs, chunk_bh=5)
+    torch.cuda.current_stream().synchronize()
+    check_device_status()
+    for r, (o, lse) in zip(runs, ref):
+        assert torch.equal(r["o_host"].view(torch.int16), o.view(torch.int16))
+        assert torch.equal(r["lse_host"], lse)
+
+
 def test_host_path_tiny_single_chunk():
     wl = WORKLOADS["tiny"]
     host = _host_inputs(wl)

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 
 SMALL = [Geometry(4, 16, 16, 32, 0.5, 2.0), Geometry(5, 3, 5, 32, 0.7, 0.3),
          Geometry(6, 8, 8, 32, 0.4, 0.1), Geometry(4, 4, 16, 64, 0.5, 2.0, theta_c=0.1, theta_m=0.2),
-         Geometry(7, 6, 7, 32, 1.0, 2.0, force_t=0)]
+         Geometry(7, 6, 7, 32, 1.0, 2.0, force_t=0), Geometry(7, 6, 16, 128, 0.4, 1.0)]
 
 
 def _gpu_mask(geom, rho1, rho2, seed, replicas=1):
@@ -59,7 +59,8 @@ def test_full_retention_is_the_candidate_set_and_replicas_repeat():
         np.testing.assert_array_equal(col[r * nnz:(r + 1) * nnz], c["col"])
 
 
-@pytest.mark.parametrize("name,rho1,rho2", [("wan13b_480p", 0.3, 0.1), ("wan14b_720p", 0.5, 0.2)])
+@pytest.mark.parametrize("name,rho1,rho2", [("wan13b_480p", 0.3, 0.1), ("wan14b_720p", 0.5, 0.2),
+                                            ("hunyuan_720p", 0.3, 0.1)])
 def test_workload_geometry_sampled(name, rho1, rho2):
     geom = WORKLOADS[name].geom
     seed = 2026
