@@ -26,7 +26,8 @@ pytestmark = pytest.mark.gpu
 
 DELTA = 1e-3
 SMALL = [Geometry(4, 8, 8, 32, 0.5, 2.0), Geometry(5, 6, 7, 32, 0.7, 0.3),
-         Geometry(4, 4, 16, 64, 0.5, 2.0, theta_c=0.1, theta_m=0.2), Geometry(6, 8, 8, 32, 0.4, 2.0, force_t=0)]
+         Geometry(4, 4, 16, 64, 0.5, 2.0, theta_c=0.1, theta_m=0.2), Geometry(6, 8, 8, 32, 0.4, 2.0, force_t=0),
+         Geometry(7, 6, 16, 128, 0.4, 1.0)]
 
 
 def _run(geom, bits, tau1, tau2, hf):
@@ -81,6 +82,31 @@ def test_small_geometries_against_the_oracle(gi, tau1, tau2, hf):
             else:
                 assert all(np.array_equal(x, y) for x, y in zip(rr, rows_gpu))
         _check_rows(geom, rows_gpu, qf, kf, tau1, tau2, list(range(nb)), f"geom {gi} b {b}")
+
+
+@pytest.mark.parametrize("D,hf", [(64, 3), (64, 4), (128, 1), (128, 3), (128, 4)])
+def test_every_fused_width(D, hf):
+    # the tensor-core tile kernel serves H_f * D <= 256, the warp-level MMA
+    # kernel the wider (128, 3) and (128, 4); every instance against the oracle
+    geom = SMALL[1]
+    B, H = 1, 4
+    tau1, tau2 = 0.5, 1.5
+    bits = random_qkv_bf16(41 + D + hf, B, H, geom.n_tokens, D, scale=1.0)
+    rp, col, st, _ = _run(geom, bits, tau1, tau2, hf)
+    F, nb = geom.frames, geom.n_blocks
+    qf = np.stack([bf16_bits_to_f64(bits["q"][0, h]) for h in range(hf)])
+    kf = np.stack([bf16_bits_to_f64(bits["k"][0, h]) for h in range(hf)])
+    for i in range(F):
+        for j in range(F):
+            if abs(i - j) < 2:
+                continue
+            n, mu, sigma, _, _, _ = DT.frame_pair_stats(geom, qf, kf, i, j)
+            if n == 0:
+                continue
+            scale = max(1.0, abs(mu), sigma)
+            assert abs(st[0, i * F + j, 0] - mu) <= 1e-5 * scale, (D, hf, i, j)
+            assert abs(st[0, i * F + j, 1] - sigma) <= 1e-5 * scale, (D, hf, i, j)
+    _check_rows(geom, csr_rows(rp, col, 0, nb), qf, kf, tau1, tau2, list(range(nb)), f"D {D} hf {hf}")
 
 
 def test_very_low_thresholds_give_the_candidate_set():
