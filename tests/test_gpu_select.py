@@ -144,3 +144,36 @@ def test_selection_without_score_export_matches(name, gamma, mode, value):
     assert torch.equal(rp1, rp2)
     n = int(rp1[-1])
     assert torch.equal(col1[:n], col2[:n])
+
+
+@pytest.mark.parametrize("mode,value", [("static", 0.2), ("dynamic", 0.85)])
+def test_every_selection_width_gives_the_same_csr(mode, value):
+    # The selection kernel is instantiated for 4, 8, 16 or 32 candidates per
+    # lane, picked from the declared longest candidate row; declaring a longer
+    # bound (clamped to Nb) picks a wider instance over the same data, which
+    # must keep exactly the same blocks.  Rows of at most 128 candidates and
+    # Nb = 576 let the same data run all four widths.
+    geom = Geometry(36, 4, 32, 8, 0.05, 0.2)
+    D = 64
+    bits = random_qkv_bf16(77, 1, 2, geom.n_tokens, D, scale=2.0)
+    q, k, _ = gpu_inputs(bits)
+    cand = abi.dynrad_build_candidates(geom)
+    nb = geom.n_blocks
+    assert nb > 512
+    real = cand["max_row"]
+    assert real <= 128
+    results = []
+    for bound in sorted({real, max(real, 129), max(real, 257), max(real, 513), nb}):
+        rp, col, scores = abi.dynrad_select_blocks(q, k, geom, dict(cand, max_row=bound), mode, value, scores=True)
+        torch.cuda.synchronize()
+        check_device_status()
+        results.append((bound, rp.cpu().numpy().astype(np.int64), col.cpu().numpy().astype(np.int64),
+                        scores.cpu().numpy()))
+    _, rp0, col0, sc0 = results[0]
+    cand_np = cand_to_numpy(cand)
+    for h in range(2):
+        assert compare_selection(mode, value, cand_np, csr_rows(rp0, col0, h, nb), sc0, h, nb, cand["nnz"]) == 0
+    for bound, rp, col, sc in results[1:]:
+        np.testing.assert_array_equal(rp, rp0, err_msg=f"bound {bound}")
+        np.testing.assert_array_equal(col[: rp0[-1]], col0[: rp0[-1]], err_msg=f"bound {bound}")
+        np.testing.assert_array_equal(sc, sc0, err_msg=f"bound {bound}")
