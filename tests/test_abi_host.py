@@ -216,6 +216,8 @@ def test_sampled_mask_argument_errors_before_launch():
     g16 = abi.make_geom(Geometry(4, 4, 4, 16, 0.5, 2.0))
     assert call(geom_=g16) == abi.DYNRAD_ERR_UNSUPPORTED
     F = geom.frames
+    assert L.dynrad_sampled_mask_workspace_min_bytes(ctypes.byref(g), 0) == 0
+    assert L.dynrad_sampled_mask_workspace_bytes(ctypes.byref(g), 0) == 0
     least = L.dynrad_sampled_mask_workspace_min_bytes(ctypes.byref(g), 100)
     # frame-pair records (56 B), two counters each plus two, thresholds, kept
     # lists, keep flags, scan partials
