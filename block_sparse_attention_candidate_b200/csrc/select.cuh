@@ -510,11 +510,14 @@ __device__ __forceinline__ uint32_t select_row(const Stage2Params& p, int I, int
       prefix = kmax & pmask;
       const int shift = top >= 7 ? top - 7 : 0;
       const uint32_t dmask = (1u << (top - shift + 1)) - 1u;
+      // 256 bins of counts (static mode) or, in dynamic mode, of weights
+      // < 2^36 split into 18-bit halves in two banks (each half's bin sum stays
+      // below 2^32 for rows of up to 2^14 candidates; two 32-bit shared atomics
+      // measured faster than one 64-bit one)
+      constexpr int kBanks = DYN ? 2 : 1;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) bins[lane * 16 + i] = 0u;
+      for (int i = 0; i < 8 * kBanks; ++i) bins[lane * 8 * kBanks + i] = 0u;
       __syncwarp();
-      // weights < 2^36 are split into 18-bit halves; each half's bin sum stays
-      // below 2^32 for rows of up to 2^14 candidates
 #pragma unroll 2
       for (int i = 0; i < ne; ++i) {
         if ((freev >> i) & 1u) {
@@ -522,9 +525,13 @@ __device__ __forceinline__ uint32_t select_row(const Stage2Params& p, int I, int
           const uint32_t k = order_key(srow[c]);
           if ((k & pmask) == prefix) {
             const uint32_t b = (k >> shift) & dmask;
-            const uint64_t w = wof(c);
-            atomicAdd(&bins[b], static_cast<uint32_t>(w & 0x3FFFFu));
-            if (w >> 18) atomicAdd(&bins[256 + b], static_cast<uint32_t>(w >> 18));
+            if constexpr (DYN) {
+              const uint64_t w = wof(c);
+              atomicAdd(&bins[b], static_cast<uint32_t>(w & 0x3FFFFu));
+              if (w >> 18) atomicAdd(&bins[256 + b], static_cast<uint32_t>(w >> 18));
+            } else {
+              atomicAdd(&bins[b], 1u);
+            }
           }
         }
       }
@@ -534,7 +541,8 @@ __device__ __forceinline__ uint32_t select_row(const Stage2Params& p, int I, int
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const uint32_t b = 255 - (lane * 8 + i);
-        loc[i] = (static_cast<uint64_t>(bins[256 + b]) << 18) + bins[b];
+        if constexpr (DYN) loc[i] = (static_cast<uint64_t>(bins[256 + b]) << 18) + bins[b];
+        else loc[i] = bins[b];
         lsum += loc[i];
       }
       const uint64_t excl = warp_excl_scan_u64(lsum, lane);
